@@ -1,0 +1,380 @@
+"""Plain fp64 CPU oracle for the Wan2.1 / Wan2.2 DiT block forward and the
+CFG-combined flow-matching Euler step.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import, call or
+execute this module: only the test suite (``tests/``), the smoke check in
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` use it. It shares no code with the CUDA library: it
+takes plain numpy arrays (the exact values handed to the GPU, upcast to
+float64) and returns float64 arrays.
+
+Sources (the pages that define what is computed):
+
+* [WALK] "Wan2.2 code walkthrough" (newtid.com/chuangyezixun/14194.html):
+  the ``WanModel`` structure snippet, the forward snippet (patch, flatten,
+  blocks), the time-projection snippet (6 x dim modulation), the
+  ``WanAttentionBlock`` core-logic snippet, the 3D RoPE snippet, the
+  self-attention snippet (global window, no causal mask) and the sampling
+  loop snippet (classifier-free guidance).
+* [DIGEST] "Wan paper deep dive" (charles2530.github.io), section
+  "Video DiT and Flow Matching": token count formula, shared AdaLN MLP with a
+  per-block bias, flow-matching path x_t = t x1 + (1-t) x0 and v = x1 - x0.
+* [TRACE] "Wan2.2 I2V inference trace" (damodev.csdn.net), section 4 "DIT":
+  token shapes and the CFG scale meaning (s = 1: prompt only).
+* [DIFFUSERS] "diffusers WanPipeline walkthrough" (huan-yin.github.io),
+  sections "3D Patchify" and "3D RoPE coordinate system".
+
+Readings taken where the pages are silent:
+
+* RoPE: every axis has its own frequency ladder omega_j = theta^(-2j/d_a),
+  d_a the axis width in real dims (t: d - 4(d//6), h = w: 2(d//6)), and
+  positions are 0-based grid indices; pairs are interleaved (2j, 2j+1).
+* QK-RMSNorm normalises the full dim-wide projection (before the head split)
+  with a learnable gain, for both self- and cross-attention q and k.
+* norm1 / norm2 carry no affine; norm3 is an affine LayerNorm. LayerNorm uses
+  the population variance with eps inside the square root.
+* Softmax scale 1/sqrt(head_dim); every Linear has a bias.
+* A query row with zero valid keys (key length 0) outputs zeros.
+
+Every function cites the passage it follows.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+F64 = np.float64
+
+
+# --------------------------------------------------------------------------
+# Token grid  ([WALK] forward snippet: Conv3d patch, flatten(2).transpose;
+# [DIGEST] token-count formula; [DIFFUSERS] "3D Patchify")
+# --------------------------------------------------------------------------
+
+def latent_grid(frames: int, height: int, width: int,
+                vae_stride=(4, 8, 8), patch=(1, 2, 2)):
+    """Token grid (F, H, W) of a clip after the VAE and the (1,2,2) patching.
+
+    The causal VAE keeps the first frame and folds every further 4 frames into
+    one latent frame ([TRACE] section 3.1 "encoder": 81 frames -> 21 latents),
+    and divides height and width by the spatial stride; the DiT patch
+    embedding then divides each axis by the patch size ([WALK] forward).
+    """
+    st, sh, sw = vae_stride
+    pt, ph, pw = patch
+    f_lat = 1 + (frames - 1) // st
+    h_lat = height // sh
+    w_lat = width // sw
+    return (f_lat // pt, h_lat // ph, w_lat // pw)
+
+
+def token_positions(F: int, H: int, W: int) -> np.ndarray:
+    """(t, h, w) grid position of every token, shape [F*H*W, 3], int64.
+
+    ``flatten(2)`` of a [C, F, H, W] tensor makes F the slowest and W the
+    fastest index ([WALK] forward snippet), so token i sits at
+    t = i // (H W), h = (i // W) mod H, w = i mod W.
+    """
+    i = np.arange(F * H * W, dtype=np.int64)
+    return np.stack([i // (H * W), (i // W) % H, i % W], axis=1)
+
+
+# --------------------------------------------------------------------------
+# 3D RoPE ([WALK] "3D RoPE" snippet; [DIFFUSERS] "3D RoPE coordinate system")
+# --------------------------------------------------------------------------
+
+def rope_axis_pairs(head_dim: int):
+    """Complex pairs given to the (t, h, w) axes: [c - 2(c//3), c//3, c//3],
+    c = head_dim / 2 ([WALK] 3D RoPE snippet, the ``split`` of the table)."""
+    if head_dim % 2:
+        raise ValueError("head_dim must be even")
+    c = head_dim // 2
+    return (c - 2 * (c // 3), c // 3, c // 3)
+
+
+def rope_omegas(head_dim: int, theta: float = 1e4) -> np.ndarray:
+    """Angular frequency of each complex pair j in [0, head_dim/2), fp64.
+
+    The table is the concatenation of one frequency ladder per axis; an axis
+    that owns p pairs (d_a = 2p real dims) has omega_j = theta^(-2j/d_a),
+    j = 0..p-1 (the plainest reading of a per-axis precomputed table split as in
+    the [WALK] snippet).
+    """
+    out = []
+    for p in rope_axis_pairs(head_dim):
+        d_a = 2 * p
+        j = np.arange(p, dtype=F64)
+        out.append(theta ** (-(2.0 * j) / d_a))
+    return np.concatenate(out)
+
+
+def rope_pair_axis(head_dim: int) -> np.ndarray:
+    """Axis (0 = t, 1 = h, 2 = w) that rotates each complex pair."""
+    pt, ph, pw = rope_axis_pairs(head_dim)
+    return np.concatenate([np.zeros(pt, np.int64), np.ones(ph, np.int64),
+                           np.full(pw, 2, np.int64)])
+
+
+def rope_table(head_dim: int, max_pos: int = 1024, theta: float = 1e4) -> np.ndarray:
+    """Precomputed table of (cos, sin) of pos * omega_j, shape
+    [max_pos, head_dim/2, 2], fp64 ([WALK]: a 1024-position table computed
+    once and sliced per grid)."""
+    ang = np.arange(max_pos, dtype=F64)[:, None] * rope_omegas(head_dim, theta)[None, :]
+    return np.stack([np.cos(ang), np.sin(ang)], axis=-1)
+
+
+def rope_apply(x: np.ndarray, grid, theta: float = 1e4,
+               positions: np.ndarray | None = None) -> np.ndarray:
+    """Rotate q or k ([L, heads, d]) by the 3D RoPE of each token.
+
+    Pair j = (x[2j], x[2j+1]) is read as the complex number x[2j] + i x[2j+1]
+    (``view_as_real(...).flatten`` in the [WALK] snippet: interleaved pairs) and is
+    multiplied by exp(i * pos_axis(j) * omega_j), where pos_axis(j) is the
+    token's t, h or w grid index for the axis that owns pair j.
+    """
+    L, n, d = x.shape
+    if positions is None:
+        positions = token_positions(*grid)
+    assert positions.shape[0] == L
+    pos = positions[:, rope_pair_axis(d)].astype(F64)           # [L, d/2]
+    ang = pos * rope_omegas(d, theta)[None, :]                  # [L, d/2]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    x = np.asarray(x, F64)
+    re = x[..., 0::2]
+    im = x[..., 1::2]
+    out = np.empty_like(x)
+    out[..., 0::2] = re * c - im * s
+    out[..., 1::2] = re * s + im * c
+    return out
+
+
+# --------------------------------------------------------------------------
+# Norms and activation ([WALK] block snippet and structure snippet)
+# --------------------------------------------------------------------------
+
+def layer_norm(x: np.ndarray, eps: float, gamma=None, beta=None) -> np.ndarray:
+    """LayerNorm over the last axis: (x - mean) / sqrt(var + eps), population
+    variance; optional affine gamma, beta (norm3)."""
+    x = np.asarray(x, F64)
+    mu = x.mean(-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(-1, keepdims=True)
+    y = (x - mu) / np.sqrt(var + eps)
+    if gamma is not None:
+        y = y * np.asarray(gamma, F64)
+    if beta is not None:
+        y = y + np.asarray(beta, F64)
+    return y
+
+
+def rms_norm(x: np.ndarray, gamma, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * gamma
+    (the optional q/k RMSNorm, ``qk_norm`` in the [WALK] structure snippet)."""
+    x = np.asarray(x, F64)
+    r = 1.0 / np.sqrt((x * x).mean(-1, keepdims=True) + eps)
+    return x * r * np.asarray(gamma, F64)
+
+
+def gelu_tanh(z: np.ndarray) -> np.ndarray:
+    """GELU, tanh form (``nn.GELU(approximate="tanh")`` in the [WALK]
+    structure snippet): 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3)))."""
+    z = np.asarray(z, F64)
+    return 0.5 * z * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3)))
+
+
+def linear(a: np.ndarray, w: np.ndarray, b) -> np.ndarray:
+    """y = a W^T + b with W stored [out, in] (``nn.Linear``)."""
+    y = np.asarray(a, F64) @ np.asarray(w, F64).T
+    if b is not None:
+        y = y + np.asarray(b, F64)
+    return y
+
+
+# --------------------------------------------------------------------------
+# Attention ([WALK] self-attention snippet: global window, no causal mask,
+# key lengths)
+# --------------------------------------------------------------------------
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+              k_len: int | None = None, scale: float | None = None) -> np.ndarray:
+    """Softmax attention of one sequence, every head.
+
+    q [Lq, n, d], k and v [Lk, n, d]; only the first ``k_len`` keys are valid.
+    o_i = sum_j softmax_j(q_i . k_j * scale) v_j with scale = 1/sqrt(d)
+    (the pages are silent; the usual default). A row with no valid key returns zeros.
+    """
+    q = np.asarray(q, F64)
+    k = np.asarray(k, F64)
+    v = np.asarray(v, F64)
+    Lq, n, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if k_len is not None:
+        k = k[:k_len]
+        v = v[:k_len]
+    if k.shape[0] == 0:
+        return np.zeros((Lq, n, v.shape[2]), F64)
+    s = np.einsum("qnd,knd->nqk", q, k) * scale
+    s = s - s.max(-1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(-1, keepdims=True)
+    return np.einsum("nqk,knd->qnd", p, v)
+
+
+# --------------------------------------------------------------------------
+# The block ([WALK] WanAttentionBlock core-logic snippet; [DIGEST] shared
+# AdaLN MLP + per-block bias)
+# --------------------------------------------------------------------------
+
+BLOCK_WEIGHT_NAMES = (
+    "modulation",
+    "wq", "bq", "wk", "bk", "wv", "bv", "wo", "bo", "gq", "gk",
+    "g3", "b3",
+    "cwq", "cbq", "cwk", "cbk", "cwv", "cbv", "cwo", "cbo", "cgq", "cgk",
+    "w1", "b1", "w2", "b2",
+)
+
+
+def block_param_count(dim: int, ffn_dim: int, biases: bool = True) -> int:
+    """Parameters of one block under this reading: four dim x dim projections
+    in each attention, two FFN matrices, their biases, the q/k gains, the
+    norm3 affine and the 6 x dim modulation bias."""
+    n = 8 * dim * dim + 2 * dim * ffn_dim
+    if biases:
+        n += 8 * dim + ffn_dim + dim          # attention + FFN biases
+        n += 4 * dim + 2 * dim + 6 * dim      # q/k gains, norm3 affine, modulation
+    return n
+
+
+def _mod(w, e0):
+    # e = (modulation + e0).chunk(6): shift, scale, gate, shift2, scale2, gate2
+    return np.asarray(w["modulation"], F64)[None] + np.asarray(e0, F64)   # [B, 6, D]
+
+
+def self_attn_kv(x, e0, w, heads, grid, eps, theta=1e4):
+    """K (RMSNorm'd, rotated) and V of the self-attention for every row of
+    every sequence: [B, L, n, d] each. Rows interact only through these."""
+    x = np.asarray(x, F64)
+    B, L, D = x.shape
+    d = D // heads
+    m = _mod(w, e0)
+    u = layer_norm(x, eps) * (1.0 + m[:, 1, None, :]) + m[:, 0, None, :]
+    k = rms_norm(linear(u, w["wk"], w["bk"]), w["gk"], eps).reshape(B, L, heads, d)
+    v = linear(u, w["wv"], w["bv"]).reshape(B, L, heads, d)
+    k = np.stack([rope_apply(k[b], grid, theta) for b in range(B)])
+    return k, v
+
+
+def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
+                       theta=1e4, kv=None, intermediates=None):
+    """Output of one WanAttentionBlock at the token rows ``rows`` of every
+    sequence: [B, len(rows), D]. Follows the [WALK] block snippet:
+
+        m = modulation + e0                        (shift, scale, gate, x2)
+        x += m2 * SelfAttn(LN(x) (1 + m1) + m0)
+        x += CrossAttn(LN_affine3(x), ctx)          (no gate, no modulation)
+        x += m5 * FFN(LN(x) (1 + m4) + m3)
+
+    SelfAttn: q, k = RMSNorm(Linear(u)), v = Linear(u); q, k rotated by the
+    3D RoPE; full softmax attention over all L tokens; output Linear.
+    CrossAttn: same without RoPE; keys/values from ctx, first ctx_lens[b] valid.
+    FFN: Linear, GELU-tanh, Linear.
+
+    Self-attention K and V need every row; everything else is row-local, so
+    only the requested rows are carried past the key/value projection.
+    ``intermediates`` (a dict) receives the per-branch outputs at those rows.
+    """
+    x = np.asarray(x, F64)
+    ctx = np.asarray(ctx, F64)
+    B, L, D = x.shape
+    T = ctx.shape[1]
+    d = D // heads
+    rows = np.asarray(rows, np.int64)
+    m = _mod(w, e0)
+    if kv is None:
+        kv = self_attn_kv(x, e0, w, heads, grid, eps, theta)
+    k_all, v_all = kv
+    pos = token_positions(*grid)[rows]
+
+    xr = x[:, rows, :].copy()                                    # [B, R, D]
+    R = rows.shape[0]
+    inter = {"o_self": [], "y_self": [], "o_cross": [], "y_cross": [], "y_ffn": [], "h": []}
+    out = np.empty_like(xr)
+    for b in range(B):
+        xb = xr[b]
+        # self-attention branch
+        u = layer_norm(xb, eps) * (1.0 + m[b, 1]) + m[b, 0]
+        q = rms_norm(linear(u, w["wq"], w["bq"]), w["gq"], eps).reshape(R, heads, d)
+        q = rope_apply(q, grid, theta, positions=pos)
+        o = attention(q, k_all[b], v_all[b]).reshape(R, D)
+        y = linear(o, w["wo"], w["bo"])
+        xb = xb + y * m[b, 2]
+        inter["o_self"].append(o)
+        inter["y_self"].append(y)
+        # cross-attention branch
+        a3 = layer_norm(xb, eps, w["g3"], w["b3"])
+        qc = rms_norm(linear(a3, w["cwq"], w["cbq"]), w["cgq"], eps).reshape(R, heads, d)
+        kc = rms_norm(linear(ctx[b], w["cwk"], w["cbk"]), w["cgk"], eps).reshape(T, heads, d)
+        vc = linear(ctx[b], w["cwv"], w["cbv"]).reshape(T, heads, d)
+        klen = T if ctx_lens is None else int(ctx_lens[b])
+        oc = attention(qc, kc, vc, k_len=klen).reshape(R, D)
+        yc = linear(oc, w["cwo"], w["cbo"])
+        xb = xb + yc
+        inter["o_cross"].append(oc)
+        inter["y_cross"].append(yc)
+        # FFN branch
+        a2 = layer_norm(xb, eps) * (1.0 + m[b, 4]) + m[b, 3]
+        h = gelu_tanh(linear(a2, w["w1"], w["b1"]))
+        yf = linear(h, w["w2"], w["b2"])
+        xb = xb + yf * m[b, 5]
+        inter["h"].append(h)
+        inter["y_ffn"].append(yf)
+        out[b] = xb
+    if intermediates is not None:
+        for key, val in inter.items():
+            intermediates[key] = np.stack(val)
+    return out
+
+
+def block_forward(x, ctx, ctx_lens, e0, w, heads, grid, eps, theta=1e4,
+                  intermediates=None):
+    """Full block output [B, L, D] (all rows)."""
+    L = np.asarray(x).shape[1]
+    return block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps,
+                              np.arange(L), theta=theta, intermediates=intermediates)
+
+
+# --------------------------------------------------------------------------
+# CFG + flow-matching Euler step ([WALK] sampling-loop snippet; [DIGEST]
+# "Video DiT and Flow Matching")
+# --------------------------------------------------------------------------
+
+def cfg_combine(v_cond, v_uncond, guide_scale: float):
+    """v = v_u + s (v_c - v_u); without an unconditional branch v = v_c."""
+    v_cond = np.asarray(v_cond, F64)
+    if v_uncond is None:
+        return v_cond
+    v_uncond = np.asarray(v_uncond, F64)
+    return v_uncond + guide_scale * (v_cond - v_uncond)
+
+
+def euler_cfg_step(x, v_cond, v_uncond, guide_scale: float,
+                   sigma: float, sigma_next: float):
+    """One explicit Euler step of the flow ODE in sigma: x + (sigma' - sigma) v."""
+    return np.asarray(x, F64) + (sigma_next - sigma) * cfg_combine(v_cond, v_uncond, guide_scale)
+
+
+def denoise_step(x_tokens, ctx_cond, ctx_uncond, ctx_lens, e0, blocks, heads, grid,
+                 eps, guide_scale, sigma, sigma_next, theta=1e4):
+    """One denoising step on the token stream: the block stack runs on the
+    same x for the conditional and the unconditional context, the two outputs
+    are combined by CFG and the Euler step moves x (there is no patch
+    embedding or head on this path)."""
+    x_tokens = np.asarray(x_tokens, F64)
+    xb = np.stack([x_tokens, x_tokens])
+    ctx = np.stack([np.asarray(ctx_cond, F64), np.asarray(ctx_uncond, F64)])
+    e = np.stack([np.asarray(e0, F64)] * 2) if np.asarray(e0).ndim == 2 else np.asarray(e0, F64)
+    for w in blocks:
+        xb = block_forward(xb, ctx, ctx_lens, e, w, heads, grid, eps, theta)
+    return euler_cfg_step(x_tokens, xb[0], xb[1], guide_scale, sigma, sigma_next)
