@@ -1,0 +1,192 @@
+/*
+ * wan.h -- C ABI of libwan: the Wan2.1 / Wan2.2 video DiT block forward and
+ * the CFG-combined flow-matching Euler step on one NVIDIA B200 (sm_100a).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - All tensor pointers are DEVICE pointers unless stated; the caller owns
+ *    every buffer. The library never allocates or frees device memory: the
+ *    block forward takes a caller-supplied workspace.
+ *  - Work is enqueued on the caller's stream (`wan_stream_t` is the same
+ *    type as `cudaStream_t`; NULL is the legacy default stream) and returns
+ *    without synchronising. Results are valid once the stream reaches them.
+ *  - Row-major, densely packed layouts. A "row" of an activation tensor is
+ *    one token. Matrices of `nn.Linear`-style projections are stored
+ *    [out_features, in_features] and applied as y = a W^T + b.
+ *  - Return value: WAN_OK (0) or a negative WAN_E* code; a human-readable
+ *    message for the calling thread is available from wan_last_error().
+ *    Argument errors are detected on the host before anything is launched.
+ *  - Every pointer must be 16-byte aligned (WAN_EALIGN otherwise).
+ *
+ * Sources (the pages that define the computation):
+ *  [WALK]   "Wan2.2 code walkthrough" (newtid.com/chuangyezixun/14194.html):
+ *           WanAttentionBlock core-logic snippet, 3D RoPE snippet,
+ *           self-attention snippet, sampling-loop (CFG) snippet.
+ *  [DIGEST] "Wan paper deep dive" (charles2530.github.io), section
+ *           "Video DiT and Flow Matching": shared AdaLN MLP with per-block
+ *           bias, flow-matching interpolation and velocity.
+ */
+#ifndef WAN_H_
+#define WAN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *wan_stream_t;
+
+/* status codes */
+#define WAN_OK            0
+#define WAN_EINVAL       -1   /* bad argument: sizes, NULL pointer, inconsistent dims   */
+#define WAN_EALIGN       -2   /* a pointer is not 16-byte aligned                       */
+#define WAN_EUNSUPPORTED -3   /* dtype / head_dim combination not implemented           */
+#define WAN_ECUDA        -4   /* a CUDA runtime or driver call failed                   */
+#define WAN_ETIMEOUT     -5   /* a kernel's bounded wait gave up (see wan_device_status) */
+
+/* element types */
+#define WAN_F32  0
+#define WAN_BF16 1
+
+/* Problem statement of one block call ([WALK]: grid sizes after the (1,2,2)
+ * patch embedding, dim, heads, ffn_dim, text length, eps). */
+typedef struct {
+  int F, H, W;      /* token grid; L = F*H*W tokens per sequence, token i at
+                       t = i/(H*W), h = (i/W)%H, w = i%W                      */
+  int dim;          /* D, model width                                         */
+  int heads;        /* n; head_dim d = dim/heads                              */
+  int ffn_dim;      /* FFN hidden width                                       */
+  int text_len;     /* T, text tokens per sequence (context rows)             */
+  float eps;        /* LayerNorm / RMSNorm epsilon (1e-6 in Wan)              */
+  int dtype;        /* WAN_F32: every matrix, bias, context and intermediate
+                       in float32 with exact fp32 FMA arithmetic.
+                       WAN_BF16: matrices, biases, context and intermediates
+                       in bfloat16, tensor-core products accumulated in fp32;
+                       norms, softmax, residual stream in fp32.              */
+} wan_dims;
+
+/* Parameters of one WanAttentionBlock ([WALK] block snippet). Pointers marked
+ * (dt) are in wan_dims.dtype, the others float32. All [dim] unless noted. */
+typedef struct {
+  const float *modulation;                 /* [6, dim] per-block bias added to e0      */
+  const void *wq, *bq, *wk, *bk, *wv, *bv; /* (dt) self-attn q/k/v: [dim,dim], [dim]   */
+  const void *wo, *bo;                     /* (dt) self-attn output projection         */
+  const float *gq, *gk;                    /* self-attn q/k RMSNorm gains              */
+  const float *g3, *b3;                    /* norm3 (affine LayerNorm) gain and bias   */
+  const void *cwq, *cbq, *cwk, *cbk, *cwv, *cbv; /* (dt) cross-attn projections       */
+  const void *cwo, *cbo;                   /* (dt) cross-attn output projection        */
+  const float *cgq, *cgk;                  /* cross-attn q/k RMSNorm gains             */
+  const void *w1, *b1;                     /* (dt) FFN in:  [ffn_dim, dim], [ffn_dim]  */
+  const void *w2, *b2;                     /* (dt) FFN out: [dim, ffn_dim], [dim]      */
+} wan_block_weights;
+
+/* Message describing the last error on the calling thread ("" if none). */
+const char *wan_last_error(void);
+
+/* wan_rope_freqs -- the precomputed 3D RoPE table ([WALK] 3D RoPE snippet:
+ * a 1024-position table split into t / h / w sections).
+ *   head_dim  d, even, 2..256. The d/2 complex pairs are split
+ *             [c - 2(c/3), c/3, c/3] (c = d/2) between the t, h, w axes; an
+ *             axis owning p pairs uses omega_j = theta^(-2j/(2p)), j < p.
+ *   max_pos   rows of the table (1024 in Wan); grid sizes must not exceed it.
+ *   theta     base (1e4 in Wan).
+ *   table     out, device, float32 [max_pos][d/2][2] = (cos, sin) of
+ *             pos * omega_j; angles are formed in fp64, stored rounded.
+ * Errors: WAN_EINVAL for odd / out-of-range head_dim, max_pos < 1, NULL. */
+int wan_rope_freqs(int head_dim, int max_pos, double theta, float *table,
+                   wan_stream_t stream);
+
+/* Bytes of workspace wan_block_forward needs for `B` sequences of `dims`
+ * (0 on invalid dims). The workspace holds, at the offsets returned by
+ * wan_block_workspace_offset, the intermediates of the last call. */
+size_t wan_block_workspace_bytes(const wan_dims *dims, int B);
+
+/* Workspace buffers (for inspection after a call; all row-major):          */
+#define WAN_WS_ACT   0  /* (dt) [B*L, dim]   last normalised branch input (FFN's)  */
+#define WAN_WS_QKV   1  /* (dt) [B*L, 3*dim] self q | k | v, q/k normalised+rotated */
+#define WAN_WS_O     2  /* (dt) [B*L, dim]   self-attention output (before W_o)     */
+#define WAN_WS_QC    3  /* (dt) [B*L, dim]   cross-attention q (normalised)         */
+#define WAN_WS_KVC   4  /* (dt) [B*T, 2*dim] cross k | v (k normalised)             */
+#define WAN_WS_OC    5  /* (dt) [B*L, dim]   cross-attention output (before W_o)    */
+#define WAN_WS_H     6  /* (dt) [B*L, ffn]   FFN hidden after GELU                  */
+#define WAN_WS_MOD   7  /* f32  [B, 6, dim]  modulation + e0                        */
+#define WAN_WS_STATS 8  /* f32  [B*L, 4]     row statistics scratch                 */
+#define WAN_WS_COUNT 9
+/* Byte offset of buffer `which` inside the workspace, or (size_t)-1. */
+size_t wan_block_workspace_offset(const wan_dims *dims, int B, int which);
+
+/* wan_block_forward -- one WanAttentionBlock on B sequences, in place on x
+ * ([WALK] WanAttentionBlock core-logic snippet):
+ *     m  = modulation + e0[b]                      (chunks m0..m5)
+ *     x += m2 * SelfAttn(LN(x) * (1 + m1) + m0)
+ *     x += CrossAttn(LN(x) * g3 + b3, ctx)         (ungated)
+ *     x += m5 * FFN(LN(x) * (1 + m4) + m3)
+ *   SelfAttn: q,k = RMSNorm_dim(a W^T + b) * gain, v = a W^T + b, q and k
+ *   rotated by 3D RoPE, softmax(q k^T / sqrt(d)) v over all L tokens of the
+ *   same sequence, output projection. CrossAttn: the same without RoPE,
+ *   keys/values from ctx, first ctx_lens[b] text tokens valid. FFN: Linear,
+ *   GELU(tanh), Linear. LayerNorm without affine uses eps inside the sqrt.
+ *
+ *   dims      problem statement; head_dim must be 128 for WAN_BF16, and one of
+ *             32, 64, 128 for WAN_F32. dim % 64 == 0, ffn_dim % 64 == 0.
+ *   B         sequences (2 for a CFG pair: same x, two contexts), >= 1.
+ *   x         in/out float32 [B, L, dim], the residual stream.
+ *   ctx       (dt) [B, T, dim] projected text tokens.
+ *   ctx_lens  device int32 [B] valid text tokens (0..T), or NULL (all T).
+ *   e0        float32 [B, 6, dim] time projection (shift, scale, gate,
+ *             shift2, scale2, gate2), shared by all blocks of a step.
+ *   w         block parameters (host struct of device pointers).
+ *   rope      table from wan_rope_freqs(head_dim, max_pos >= max(F,H,W)).
+ *   rope_max_pos  rows in that table.
+ *   workspace device buffer of ws_bytes >= wan_block_workspace_bytes().
+ * Errors: WAN_EINVAL (dims, NULLs, small workspace, grid beyond the table),
+ * WAN_EUNSUPPORTED (head_dim/dtype), WAN_EALIGN, WAN_ECUDA. */
+int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx,
+                      const int *ctx_lens, const float *e0,
+                      const wan_block_weights *w, const float *rope,
+                      int rope_max_pos, void *workspace, size_t ws_bytes,
+                      wan_stream_t stream);
+
+/* wan_attention -- softmax attention, non-causal, every head
+ * ([WALK] self-attention snippet: global window, key lengths).
+ *   B, heads, Lq, Lk, head_dim   sizes (head_dim 128 for WAN_BF16; 32, 64
+ *                                or 128 for WAN_F32).
+ *   q         (dt) [B, Lq, heads, head_dim]; k, v (dt) [B, Lk, heads, head_dim].
+ *   o         out (dt) [B, Lq, heads, head_dim]; must not alias q, k or v.
+ *   k_lens    device int32 [B] valid keys per sequence (0..Lk), or NULL (Lk);
+ *             a sequence with 0 valid keys gets o = 0.
+ *   scale     logit scale; pass 0 for 1/sqrt(head_dim).
+ *   grid      HOST int[3] = (F, H, W) with F*H*W == Lq == Lk: q and k are
+ *             first rotated IN PLACE by the 3D RoPE of their token index
+ *             (using `rope`, rope_max_pos rows); NULL: q, k are read only.
+ *   rope, rope_max_pos  ignored when grid is NULL. */
+int wan_attention(int B, int heads, int Lq, int Lk, int head_dim, int dtype,
+                  void *q, void *k, const void *v, void *o,
+                  const int *k_lens, float scale, const int *grid,
+                  const float *rope, int rope_max_pos, wan_stream_t stream);
+
+/* wan_euler_cfg_step -- classifier-free guidance followed by one explicit
+ * Euler step of the flow-matching ODE ([WALK] sampling-loop snippet;
+ * [DIGEST] "Video DiT and Flow Matching"):
+ *     v = v_uncond + guide_scale * (v_cond - v_uncond)   (v = v_cond if v_uncond NULL)
+ *     x = x + (sigma_next - sigma) * v
+ *   x         in/out float32 [n].
+ *   v_cond, v_uncond  [n] in v_dtype (WAN_F32 or WAN_BF16); may alias each
+ *             other, not x.
+ * Arithmetic in fp32 (one FMA chain per element). n may be 0. */
+int wan_euler_cfg_step(float *x, const void *v_cond, const void *v_uncond,
+                       int v_dtype, size_t n, float guide_scale, float sigma,
+                       float sigma_next, wan_stream_t stream);
+
+/* wan_device_status -- synchronise `stream`, then report and clear the
+ * library's device-side watchdog word for the current device: WAN_OK, or
+ * WAN_ETIMEOUT if a kernel gave up a bounded wait since the last call (its
+ * outputs are then invalid), or WAN_ECUDA if the stream holds a CUDA error. */
+int wan_device_status(wan_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WAN_H_ */

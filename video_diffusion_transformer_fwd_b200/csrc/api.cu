@@ -1,0 +1,338 @@
+// C ABI of libwan: argument checking, workspace layout and the launch
+// sequence of one WanAttentionBlock ("Wan2.2 code walkthrough" (newtid.com),
+// WanAttentionBlock core-logic snippet) and the CFG-Euler step (sampling-loop
+// snippet; "Wan paper deep dive" (charles2530.github.io), "Video DiT and
+// Flow Matching").
+#include "common.cuh"
+
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <climits>
+#include <mutex>
+
+namespace wan {
+
+static thread_local char g_msg[512] = "";
+
+int set_error(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_error(cudaError_t e, const char *what) {
+  return set_error(WAN_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Watchdog word: kernels with bounded waits write a nonzero code here when a
+// wait runs out (they never trap).
+__device__ int g_watchdog_word;
+
+int *watchdog_ptr() {
+  static int *ptrs[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_watchdog_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int *>(p);
+  }
+  return ptrs[dev];
+}
+
+// ---------------------------------------------------------------- dispatch
+static int run_gemm(const GemmArgs &g, int dtype, cudaStream_t s) {
+  if (dtype == WAN_BF16 && gemm_tc_supported(g)) return gemm_tc(g, s);
+  return gemm_simt(g, dtype, s);
+}
+
+static int run_attention(const AttnArgs &a, int dtype, cudaStream_t s) {
+  if (dtype == WAN_BF16 && attention_tc_supported(a)) return attention_tc(a, s);
+  return attention_simt(a, dtype, s);
+}
+
+// ---------------------------------------------------------------- workspace
+struct WsLayout {
+  size_t off[WAN_WS_COUNT];
+  size_t total;
+};
+
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+static int check_dims(const wan_dims *d, int B) {
+  if (!d) return set_error(WAN_EINVAL, "dims is NULL");
+  if (B < 0) return set_error(WAN_EINVAL, "B=%d < 0", B);
+  if (d->F < 1 || d->H < 1 || d->W < 1) return set_error(WAN_EINVAL, "grid %dx%dx%d", d->F, d->H, d->W);
+  if (d->dim < 64 || d->dim % 64) return set_error(WAN_EINVAL, "dim %d must be a positive multiple of 64", d->dim);
+  if (d->dim > 8192) return set_error(WAN_EUNSUPPORTED, "dim %d > 8192", d->dim);
+  if (d->heads < 1 || d->dim % d->heads) return set_error(WAN_EINVAL, "dim %d not divisible by heads %d", d->dim, d->heads);
+  if (d->ffn_dim < 64 || d->ffn_dim % 64) return set_error(WAN_EINVAL, "ffn_dim %d must be a positive multiple of 64", d->ffn_dim);
+  if (d->text_len < 0) return set_error(WAN_EINVAL, "text_len %d < 0", d->text_len);
+  if (!(d->eps >= 0.f)) return set_error(WAN_EINVAL, "eps must be >= 0");
+  if (d->dtype != WAN_F32 && d->dtype != WAN_BF16) return set_error(WAN_EUNSUPPORTED, "dtype %d", d->dtype);
+  const int hd = d->dim / d->heads;
+  if (d->dtype == WAN_BF16 && hd != 128) return set_error(WAN_EUNSUPPORTED, "bf16 path needs head_dim 128 (got %d)", hd);
+  if (d->dtype == WAN_F32 && hd != 32 && hd != 64 && hd != 128)
+    return set_error(WAN_EUNSUPPORTED, "fp32 path needs head_dim 32, 64 or 128 (got %d)", hd);
+  const long long L = (long long)d->F * d->H * d->W;
+  if (L * (long long)(B > 0 ? B : 1) > INT_MAX / 4) return set_error(WAN_EINVAL, "B*L too large");
+  if ((long long)d->text_len * (B > 0 ? B : 1) > INT_MAX / 4) return set_error(WAN_EINVAL, "B*T too large");
+  return WAN_OK;
+}
+
+static WsLayout layout_of(const wan_dims *d, int B) {
+  WsLayout w;
+  const size_t es = dtype_size(d->dtype);
+  const size_t BL = (size_t)B * d->F * d->H * d->W, D = d->dim, T = d->text_len, Fh = d->ffn_dim;
+  const size_t sz[WAN_WS_COUNT] = {
+      BL * D * es,            // ACT
+      BL * 3 * D * es,        // QKV
+      BL * D * es,            // O
+      BL * D * es,            // QC
+      (size_t)B * T * 2 * D * es,  // KVC
+      BL * D * es,            // OC
+      BL * Fh * es,           // H
+      (size_t)B * 6 * D * 4,  // MOD
+      BL * 4 * 4,             // STATS
+  };
+  size_t o = 0;
+  for (int i = 0; i < WAN_WS_COUNT; ++i) {
+    w.off[i] = o;
+    o += align256(sz[i]);
+  }
+  w.total = o;
+  return w;
+}
+
+}  // namespace wan
+
+using namespace wan;
+
+extern "C" {
+
+const char *wan_last_error(void) { return g_msg; }
+
+int wan_rope_freqs(int head_dim, int max_pos, double theta, float *table, wan_stream_t stream) {
+  g_msg[0] = 0;
+  if (head_dim < 2 || head_dim > 256 || head_dim % 2) return set_error(WAN_EINVAL, "head_dim %d", head_dim);
+  if (max_pos < 1) return set_error(WAN_EINVAL, "max_pos %d", max_pos);
+  if (!(theta > 0.0)) return set_error(WAN_EINVAL, "theta must be > 0");
+  if (!table) return set_error(WAN_EINVAL, "table is NULL");
+  if (!aligned16(table)) return set_error(WAN_EALIGN, "table not 16-byte aligned");
+  return launch_rope_table(head_dim, max_pos, theta, table, (cudaStream_t)stream);
+}
+
+size_t wan_block_workspace_bytes(const wan_dims *dims, int B) {
+  if (check_dims(dims, B) != WAN_OK) return 0;
+  return layout_of(dims, B).total;
+}
+
+size_t wan_block_workspace_offset(const wan_dims *dims, int B, int which) {
+  if (check_dims(dims, B) != WAN_OK || which < 0 || which >= WAN_WS_COUNT) return (size_t)-1;
+  return layout_of(dims, B).off[which];
+}
+
+int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, const int *ctx_lens,
+                      const float *e0, const wan_block_weights *w, const float *rope,
+                      int rope_max_pos, void *workspace, size_t ws_bytes, wan_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_dims(dims, B);
+  if (rc) return rc;
+  if (B == 0) return WAN_OK;
+  if (!w) return set_error(WAN_EINVAL, "weights is NULL");
+  const wan_dims &d = *dims;
+  const int L = d.F * d.H * d.W, D = d.dim, T = d.text_len, Fh = d.ffn_dim, hd = D / d.heads;
+  const int dt = d.dtype;
+  const size_t es = dtype_size(dt);
+  cudaStream_t s = (cudaStream_t)stream;
+
+  const void *ptrs[] = {x, e0, rope, workspace, w->modulation, w->wq, w->bq, w->wk, w->bk, w->wv,
+                        w->bv, w->wo, w->bo, w->gq, w->gk, w->g3, w->b3, w->cwq, w->cbq, w->cwk,
+                        w->cbk, w->cwv, w->cbv, w->cwo, w->cbo, w->cgq, w->cgk, w->w1, w->b1,
+                        w->w2, w->b2};
+  for (size_t i = 0; i < sizeof(ptrs) / sizeof(ptrs[0]); ++i) {
+    if (!ptrs[i]) return set_error(WAN_EINVAL, "pointer argument #%zu is NULL", i);
+    if (!aligned16(ptrs[i])) return set_error(WAN_EALIGN, "pointer argument #%zu not 16-byte aligned", i);
+  }
+  if (T > 0 && !ctx) return set_error(WAN_EINVAL, "ctx is NULL");
+  if (ctx && !aligned16(ctx)) return set_error(WAN_EALIGN, "ctx not 16-byte aligned");
+  if (ctx_lens && !aligned16(ctx_lens)) return set_error(WAN_EALIGN, "ctx_lens not 16-byte aligned");
+  const int gmax = d.F > d.H ? (d.F > d.W ? d.F : d.W) : (d.H > d.W ? d.H : d.W);
+  if (rope_max_pos < gmax) return set_error(WAN_EINVAL, "rope table has %d rows, grid needs %d", rope_max_pos, gmax);
+  const WsLayout lay = layout_of(dims, B);
+  if (ws_bytes < lay.total) return set_error(WAN_EINVAL, "workspace %zu bytes < %zu needed", ws_bytes, lay.total);
+
+  char *ws = static_cast<char *>(workspace);
+  void *act = ws + lay.off[WAN_WS_ACT];
+  char *qkv = ws + lay.off[WAN_WS_QKV];
+  void *o = ws + lay.off[WAN_WS_O];
+  void *qc = ws + lay.off[WAN_WS_QC];
+  char *kvc = ws + lay.off[WAN_WS_KVC];
+  void *oc = ws + lay.off[WAN_WS_OC];
+  void *hbuf = ws + lay.off[WAN_WS_H];
+  float *mod = reinterpret_cast<float *>(ws + lay.off[WAN_WS_MOD]);
+  const int BL = B * L;
+
+  // m = modulation + e0  (shift, scale, gate, shift2, scale2, gate2)
+  if ((rc = launch_mod_combine(w->modulation, e0, mod, B, D, s))) return rc;
+
+  // ---- self-attention branch: x += m2 * Wo . Attn(RoPE(RMSNorm(q,k)), v)
+  if ((rc = launch_layernorm_mod(x, act, dt, BL, D, L, mod, 0, 1, nullptr, nullptr, d.eps, s))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = 3 * D; g.K = D; g.A = act; g.lda = D;
+    g.Bseg[0] = w->wq; g.Bseg[1] = w->wk; g.Bseg[2] = w->wv;
+    g.bias[0] = w->bq; g.bias[1] = w->bk; g.bias[2] = w->bv;
+    g.segN = D; g.nseg = 3; g.epi = EPI_STORE; g.C = qkv; g.ldc = 3 * D;
+    if ((rc = run_gemm(g, dt, s))) return rc;
+  }
+  if ((rc = launch_rmsnorm_rope(qkv, dt, BL, 3 * D, D, hd, w->gq, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s))) return rc;
+  if ((rc = launch_rmsnorm_rope(qkv + D * es, dt, BL, 3 * D, D, hd, w->gk, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s))) return rc;
+  {
+    AttnArgs a = {};
+    a.B = B; a.heads = d.heads; a.Lq = L; a.Lk = L; a.d = hd;
+    a.q = qkv; a.ldq = 3 * D; a.k = qkv + D * es; a.ldk = 3 * D; a.v = qkv + 2 * D * es; a.ldv = 3 * D;
+    a.o = o; a.ldo = D; a.k_lens = nullptr; a.scale = 1.0f / sqrtf((float)hd);
+    if ((rc = run_attention(a, dt, s))) return rc;
+  }
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = D; g.A = o; g.lda = D;
+    g.Bseg[0] = w->wo; g.bias[0] = w->bo; g.segN = D; g.nseg = 1;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = mod + 2 * D; g.gate_stride = 6 * D; g.rows_per_gate = L;
+    if ((rc = run_gemm(g, dt, s))) return rc;
+  }
+
+  // ---- cross-attention branch (ungated): x += Wco . Attn(q(norm3 x), k(ctx), v(ctx))
+  if ((rc = launch_layernorm_mod(x, act, dt, BL, D, L, nullptr, 0, 0, w->g3, w->b3, d.eps, s))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = D; g.A = act; g.lda = D;
+    g.Bseg[0] = w->cwq; g.bias[0] = w->cbq; g.segN = D; g.nseg = 1;
+    g.epi = EPI_STORE; g.C = qc; g.ldc = D;
+    if ((rc = run_gemm(g, dt, s))) return rc;
+  }
+  if ((rc = launch_rmsnorm_rope(qc, dt, BL, D, D, hd, w->cgq, d.eps, nullptr, 0, 1, 1, 1, s))) return rc;
+  if (T > 0) {
+    GemmArgs g = {};
+    g.M = B * T; g.N = 2 * D; g.K = D; g.A = ctx; g.lda = D;
+    g.Bseg[0] = w->cwk; g.Bseg[1] = w->cwv; g.bias[0] = w->cbk; g.bias[1] = w->cbv;
+    g.segN = D; g.nseg = 2; g.epi = EPI_STORE; g.C = kvc; g.ldc = 2 * D;
+    if ((rc = run_gemm(g, dt, s))) return rc;
+    if ((rc = launch_rmsnorm_rope(kvc, dt, B * T, 2 * D, D, hd, w->cgk, d.eps, nullptr, 0, 1, 1, 1, s))) return rc;
+  }
+  {
+    AttnArgs a = {};
+    a.B = B; a.heads = d.heads; a.Lq = L; a.Lk = T; a.d = hd;
+    a.q = qc; a.ldq = D; a.k = kvc; a.ldk = 2 * D; a.v = kvc + D * es; a.ldv = 2 * D;
+    a.o = oc; a.ldo = D; a.k_lens = ctx_lens; a.scale = 1.0f / sqrtf((float)hd);
+    if ((rc = run_attention(a, dt, s))) return rc;
+  }
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = D; g.A = oc; g.lda = D;
+    g.Bseg[0] = w->cwo; g.bias[0] = w->cbo; g.segN = D; g.nseg = 1;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = nullptr; g.rows_per_gate = L;
+    if ((rc = run_gemm(g, dt, s))) return rc;
+  }
+
+  // ---- FFN branch: x += m5 * W2 . gelu_tanh(W1 . (LN(x)(1 + m4) + m3))
+  if ((rc = launch_layernorm_mod(x, act, dt, BL, D, L, mod, 3, 4, nullptr, nullptr, d.eps, s))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = Fh; g.K = D; g.A = act; g.lda = D;
+    g.Bseg[0] = w->w1; g.bias[0] = w->b1; g.segN = Fh; g.nseg = 1;
+    g.epi = EPI_GELU; g.C = hbuf; g.ldc = Fh;
+    if ((rc = run_gemm(g, dt, s))) return rc;
+  }
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = Fh; g.A = hbuf; g.lda = Fh;
+    g.Bseg[0] = w->w2; g.bias[0] = w->b2; g.segN = D; g.nseg = 1;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = mod + 5 * D; g.gate_stride = 6 * D; g.rows_per_gate = L;
+    if ((rc = run_gemm(g, dt, s))) return rc;
+  }
+  return WAN_OK;
+}
+
+int wan_attention(int B, int heads, int Lq, int Lk, int head_dim, int dtype, void *q, void *k,
+                  const void *v, void *o, const int *k_lens, float scale, const int *grid,
+                  const float *rope, int rope_max_pos, wan_stream_t stream) {
+  g_msg[0] = 0;
+  if (B < 0 || heads < 1 || Lq < 0 || Lk < 0) return set_error(WAN_EINVAL, "bad sizes");
+  if (dtype != WAN_F32 && dtype != WAN_BF16) return set_error(WAN_EUNSUPPORTED, "dtype %d", dtype);
+  if (dtype == WAN_BF16 && head_dim != 128) return set_error(WAN_EUNSUPPORTED, "bf16 attention needs head_dim 128");
+  if (dtype == WAN_F32 && head_dim != 32 && head_dim != 64 && head_dim != 128)
+    return set_error(WAN_EUNSUPPORTED, "fp32 attention needs head_dim 32, 64 or 128");
+  if ((long long)B * Lq * heads * head_dim > (long long)INT_MAX * 8 || (long long)B * Lq > INT_MAX / 4 ||
+      (long long)B * Lk > INT_MAX / 4)
+    return set_error(WAN_EINVAL, "sizes too large");
+  if (B == 0 || Lq == 0) return WAN_OK;
+  if (!q || !o || (Lk > 0 && (!k || !v))) return set_error(WAN_EINVAL, "NULL tensor");
+  const void *ps[] = {q, k, v, o, k_lens};
+  for (const void *p : ps)
+    if (p && !aligned16(p)) return set_error(WAN_EALIGN, "pointer not 16-byte aligned");
+  const size_t es = dtype_size(dtype);
+  const size_t qbytes = (size_t)B * Lq * heads * head_dim * es;
+  const size_t kbytes = (size_t)B * Lk * heads * head_dim * es;
+  const char *oc = static_cast<const char *>(o);
+  auto overlap = [&](const void *p, size_t n) {
+    const char *c = static_cast<const char *>(p);
+    return p && c < oc + qbytes && oc < c + n;
+  };
+  if (overlap(q, qbytes) || overlap(k, kbytes) || overlap(v, kbytes)) return set_error(WAN_EINVAL, "o aliases q, k or v");
+  cudaStream_t s = (cudaStream_t)stream;
+  const int D = heads * head_dim;
+  int rc;
+  if (grid) {
+    const int F = grid[0], H = grid[1], W = grid[2];
+    if (q == k) return set_error(WAN_EINVAL, "q and k must be distinct buffers when grid is given");
+    if (F < 1 || H < 1 || W < 1 || (long long)F * H * W != Lq || Lq != Lk)
+      return set_error(WAN_EINVAL, "grid %dx%dx%d does not match Lq=%d Lk=%d", F, H, W, Lq, Lk);
+    const int gmax = F > H ? (F > W ? F : W) : (H > W ? H : W);
+    if (!rope || rope_max_pos < gmax) return set_error(WAN_EINVAL, "rope table missing or too short");
+    if (!aligned16(rope)) return set_error(WAN_EALIGN, "rope not 16-byte aligned");
+    if ((rc = launch_rope_only(q, dtype, B * Lq, D, D, head_dim, rope, rope_max_pos, F, H, W, s))) return rc;
+    if ((rc = launch_rope_only(k, dtype, B * Lk, D, D, head_dim, rope, rope_max_pos, F, H, W, s))) return rc;
+  }
+  AttnArgs a = {};
+  a.B = B; a.heads = heads; a.Lq = Lq; a.Lk = Lk; a.d = head_dim;
+  a.q = q; a.ldq = D; a.k = k; a.ldk = D; a.v = v; a.ldv = D; a.o = o; a.ldo = D;
+  a.k_lens = k_lens; a.scale = scale != 0.f ? scale : 1.0f / sqrtf((float)head_dim);
+  return run_attention(a, dtype, s);
+}
+
+int wan_euler_cfg_step(float *x, const void *v_cond, const void *v_uncond, int v_dtype, size_t n,
+                       float guide_scale, float sigma, float sigma_next, wan_stream_t stream) {
+  g_msg[0] = 0;
+  if (n == 0) return WAN_OK;
+  if (!x || !v_cond) return set_error(WAN_EINVAL, "NULL tensor");
+  if (v_dtype != WAN_F32 && v_dtype != WAN_BF16) return set_error(WAN_EUNSUPPORTED, "v_dtype %d", v_dtype);
+  if (!aligned16(x) || !aligned16(v_cond) || (v_uncond && !aligned16(v_uncond)))
+    return set_error(WAN_EALIGN, "pointer not 16-byte aligned");
+  return launch_euler_cfg(x, v_cond, v_uncond, v_dtype, n, guide_scale, sigma_next - sigma,
+                          (cudaStream_t)stream);
+}
+
+int wan_device_status(wan_stream_t stream) {
+  g_msg[0] = 0;
+  WAN_TRY_CUDA(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize");
+  int *p = watchdog_ptr();
+  if (!p) return set_error(WAN_ECUDA, "watchdog symbol unavailable");
+  int v = 0;
+  WAN_TRY_CUDA(cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost), "read watchdog");
+  if (v != 0) {
+    const int zero = 0;
+    WAN_TRY_CUDA(cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice), "clear watchdog");
+    return set_error(WAN_ETIMEOUT, "a kernel gave up a bounded wait (code %d)", v);
+  }
+  return WAN_OK;
+}
+
+}  // extern "C"

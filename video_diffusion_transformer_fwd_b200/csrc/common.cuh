@@ -1,0 +1,154 @@
+// Shared helpers of libwan (host + device). Internal header.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/wan.h"
+
+namespace wan {
+
+// ---------------------------------------------------------------- errors
+int set_error(int code, const char *fmt, ...);
+int cuda_error(cudaError_t e, const char *what);
+// Device address of the library's watchdog word on the current device
+// (set to a nonzero code by a kernel that gave up a bounded wait).
+int *watchdog_ptr();
+
+#define WAN_TRY_CUDA(call, what)                                        \
+  do {                                                                  \
+    cudaError_t e_ = (call);                                            \
+    if (e_ != cudaSuccess) return ::wan::cuda_error(e_, what);          \
+  } while (0)
+
+#define WAN_CHECK_LAUNCH(what)                                          \
+  do {                                                                  \
+    cudaError_t e_ = cudaGetLastError();                                \
+    if (e_ != cudaSuccess) return ::wan::cuda_error(e_, what);          \
+  } while (0)
+
+// ---------------------------------------------------------------- element access
+template <typename T> struct ElemIO;
+template <> struct ElemIO<float> {
+  static __device__ __forceinline__ float load(const float *p) { return *p; }
+  static __device__ __forceinline__ void store(float *p, float v) { *p = v; }
+};
+template <> struct ElemIO<__nv_bfloat16> {
+  static __device__ __forceinline__ float load(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+  static __device__ __forceinline__ void store(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+};
+
+// load 4 consecutive elements (16-byte aligned for float, 8-byte for bf16)
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+  uint2 u = *reinterpret_cast<const uint2 *>(p);
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&u.x);
+  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&u.y);
+  float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+__device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t *>(&a);
+  u.y = *reinterpret_cast<uint32_t *>(&b);
+  *reinterpret_cast<uint2 *>(p) = u;
+}
+
+// GELU, tanh form: 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3)))
+__device__ __forceinline__ float gelu_tanh(float z) {
+  const float k0 = 0.7978845608028654f;   // sqrt(2/pi)
+  const float k1 = 0.044715f;
+  return 0.5f * z * (1.0f + tanhf(k0 * (z + k1 * z * z * z)));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide sum; `red` is shared scratch of >= 32 floats. All threads get it.
+__device__ __forceinline__ float block_sum(float v, float *red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float t = (lane < nw) ? red[lane] : 0.f;
+  return warp_sum(t);
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t dtype_size(int dt) { return dt == WAN_BF16 ? 2 : 4; }
+
+// ---------------------------------------------------------------- internal kernels API
+
+enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2 };
+
+// C = A B^T (+ bias) with a fused epilogue. A [M,K] row-major (lda),
+// B given as up to 3 row-major segments [segN, K] (ldb = K) stacked along N,
+// so one call can multiply by [Wq; Wk; Wv]. bias per segment [segN] (or NULL).
+//   EPI_STORE: C[m,n] = acc + bias
+//   EPI_GELU:  C[m,n] = gelu_tanh(acc + bias)
+//   EPI_RESID: X[m,n] += g * (acc + bias), g = gate[(m / rows_per_gate) *
+//              gate_stride + n] or 1 when gate == NULL  (X float32, ldx)
+struct GemmArgs {
+  int M, N, K;
+  const void *A; int lda;
+  const void *Bseg[3]; const void *bias[3]; int segN; int nseg;
+  int epi;
+  void *C; int ldc;
+  float *X; int ldx;
+  const float *gate; int gate_stride; int rows_per_gate;
+};
+
+int gemm_simt(const GemmArgs &g, int dtype, cudaStream_t s);
+int gemm_tc(const GemmArgs &g, cudaStream_t s);           // bf16 tcgen05 path
+bool gemm_tc_supported(const GemmArgs &g);
+
+// Attention over rows of strided matrices. Sequence b, row r of q is at
+// q + (b*Lq + r)*ldq + head*d (likewise k, v with Lk, o with Lq).
+struct AttnArgs {
+  int B, heads, Lq, Lk, d;
+  const void *q; int ldq;
+  const void *k; int ldk;
+  const void *v; int ldv;
+  void *o; int ldo;
+  const int *k_lens;      // device [B] or NULL
+  float scale;
+};
+int attention_simt(const AttnArgs &a, int dtype, cudaStream_t s);
+int attention_tc(const AttnArgs &a, cudaStream_t s);      // bf16, d = 128
+bool attention_tc_supported(const AttnArgs &a);
+
+// Elementwise / row kernels (elementwise.cu)
+int launch_mod_combine(const float *modulation, const float *e0, float *mod, int B, int D,
+                       cudaStream_t s);
+// out[r] = LN(x[r]) * (1 + mod[b][scale_chunk]) + mod[b][shift_chunk]     (affine == NULL)
+// out[r] = LN(x[r]) * g + beta                                            (affine gain g)
+int launch_layernorm_mod(const float *x, void *out, int dtype, int rows, int D, int rows_per_b,
+                         const float *mod, int shift_chunk, int scale_chunk,
+                         const float *g, const float *beta, float eps, cudaStream_t s);
+// In place on rows of a strided matrix: v = RMSNorm_D(v) * gain, then the 3D
+// RoPE of token (r % L) when rope != NULL.
+int launch_rmsnorm_rope(void *p, int dtype, int rows, int ld, int D, int head_dim,
+                        const float *gain, float eps, const float *rope, int rope_max_pos,
+                        int F, int H, int W, cudaStream_t s);
+// In place 3D RoPE only (no norm), rows of a [rows, heads*d] strided matrix.
+int launch_rope_only(void *p, int dtype, int rows, int ld, int D, int head_dim,
+                     const float *rope, int rope_max_pos, int F, int H, int W, cudaStream_t s);
+int launch_rope_table(int head_dim, int max_pos, double theta, float *table, cudaStream_t s);
+int launch_euler_cfg(float *x, const void *vc, const void *vu, int vdt, size_t n, float scale,
+                     float dt, cudaStream_t s);
+
+}  // namespace wan

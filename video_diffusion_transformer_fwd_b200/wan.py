@@ -1,0 +1,239 @@
+"""ctypes binding of libwan (the C ABI declared in include/wan.h).
+
+Argument marshalling only: the raw entry points keep the C names
+(``wan_block_forward`` and so on) and take integer device addresses; the
+torch helpers below them pull ``data_ptr()`` and the current CUDA stream out
+of tensors and raise ``WanError`` on a nonzero status. Every computation runs
+inside the library. Loading fails loudly if ``libwan.so`` has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libwan.so")
+
+WAN_OK, WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED, WAN_ECUDA, WAN_ETIMEOUT = 0, -1, -2, -3, -4, -5
+WAN_F32, WAN_BF16 = 0, 1
+(WAN_WS_ACT, WAN_WS_QKV, WAN_WS_O, WAN_WS_QC, WAN_WS_KVC, WAN_WS_OC, WAN_WS_H, WAN_WS_MOD,
+ WAN_WS_STATS) = range(9)
+STATUS_NAMES = {0: "WAN_OK", -1: "WAN_EINVAL", -2: "WAN_EALIGN", -3: "WAN_EUNSUPPORTED",
+                -4: "WAN_ECUDA", -5: "WAN_ETIMEOUT"}
+
+
+class WanError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class wan_dims(ctypes.Structure):
+    _fields_ = [("F", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("dim", ctypes.c_int), ("heads", ctypes.c_int), ("ffn_dim", ctypes.c_int),
+                ("text_len", ctypes.c_int), ("eps", ctypes.c_float), ("dtype", ctypes.c_int)]
+
+
+WEIGHT_FIELDS = ("modulation", "wq", "bq", "wk", "bk", "wv", "bv", "wo", "bo", "gq", "gk",
+                 "g3", "b3", "cwq", "cbq", "cwk", "cbk", "cwv", "cbv", "cwo", "cbo",
+                 "cgq", "cgk", "w1", "b1", "w2", "b2")
+
+
+class wan_block_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
+
+
+_c_int, _vp, _sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
+
+_SIGS = {
+    "wan_last_error": (ctypes.c_char_p, []),
+    "wan_rope_freqs": (_c_int, [_c_int, _c_int, ctypes.c_double, _vp, _vp]),
+    "wan_block_workspace_bytes": (_sz, [ctypes.POINTER(wan_dims), _c_int]),
+    "wan_block_workspace_offset": (_sz, [ctypes.POINTER(wan_dims), _c_int, _c_int]),
+    "wan_block_forward": (_c_int, [ctypes.POINTER(wan_dims), _c_int, _vp, _vp, _vp, _vp,
+                                   ctypes.POINTER(wan_block_weights), _vp, _c_int, _vp, _sz, _vp]),
+    "wan_attention": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
+                               _vp, ctypes.c_float, ctypes.POINTER(ctypes.c_int), _vp, _c_int, _vp]),
+    "wan_euler_cfg_step": (_c_int, [_vp, _vp, _vp, _c_int, _sz, ctypes.c_float, ctypes.c_float,
+                                    ctypes.c_float, _vp]),
+    "wan_device_status": (_c_int, [_vp]),
+}
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libwan.so (raises if it is missing: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libwan.so not built at {path}; run "
+                           "`python -m video_diffusion_transformer_fwd_b200.build_lib`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def wan_last_error() -> bytes:
+    return load().wan_last_error()
+
+
+def last_error() -> str:
+    return wan_last_error().decode()
+
+
+def check(rc: int):
+    if rc != WAN_OK:
+        raise WanError(rc, last_error())
+
+
+# ---------------------------------------------------------------- raw C entry points
+def wan_rope_freqs(head_dim, max_pos, theta, table, stream):
+    return load().wan_rope_freqs(head_dim, max_pos, theta, table, stream)
+
+
+def wan_block_workspace_bytes(dims, B):
+    return load().wan_block_workspace_bytes(ctypes.byref(dims), B)
+
+
+def wan_block_workspace_offset(dims, B, which):
+    return load().wan_block_workspace_offset(ctypes.byref(dims), B, which)
+
+
+def wan_block_forward(dims, B, x, ctx, ctx_lens, e0, weights, rope, rope_max_pos, workspace,
+                      ws_bytes, stream):
+    return load().wan_block_forward(ctypes.byref(dims), B, x, ctx, ctx_lens, e0,
+                                    ctypes.byref(weights), rope, rope_max_pos, workspace,
+                                    ws_bytes, stream)
+
+
+def wan_attention(B, heads, Lq, Lk, head_dim, dtype, q, k, v, o, k_lens, scale, grid, rope,
+                  rope_max_pos, stream):
+    g = None if grid is None else (ctypes.c_int * 3)(*grid)
+    return load().wan_attention(B, heads, Lq, Lk, head_dim, dtype, q, k, v, o, k_lens, scale,
+                                g, rope, rope_max_pos, stream)
+
+
+def wan_euler_cfg_step(x, v_cond, v_uncond, v_dtype, n, guide_scale, sigma, sigma_next, stream):
+    return load().wan_euler_cfg_step(x, v_cond, v_uncond, v_dtype, n, guide_scale, sigma,
+                                     sigma_next, stream)
+
+
+def wan_device_status(stream):
+    return load().wan_device_status(stream)
+
+
+# ---------------------------------------------------------------- torch helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream=None):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return WAN_BF16
+    if t.dtype == torch.float32:
+        return WAN_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def make_dims(F, H, W, dim, heads, ffn_dim, text_len, eps=1e-6, dtype="bf16") -> wan_dims:
+    code = {"bf16": WAN_BF16, "f32": WAN_F32}[dtype] if isinstance(dtype, str) else int(dtype)
+    return wan_dims(F, H, W, dim, heads, ffn_dim, text_len, eps, code)
+
+
+def dims_of(cfg) -> wan_dims:
+    return make_dims(cfg.F, cfg.H, cfg.W, cfg.dim, cfg.heads, cfg.ffn_dim, cfg.text_len,
+                     cfg.eps, cfg.dtype)
+
+
+def make_weights(w: dict) -> wan_block_weights:
+    for n in WEIGHT_FIELDS:
+        if not w[n].is_contiguous():
+            raise ValueError(f"weight {n} must be contiguous")
+    return wan_block_weights(*[w[n].data_ptr() for n in WEIGHT_FIELDS])
+
+
+def rope_freqs(head_dim, max_pos=1024, theta=1e4, device="cuda", stream=None):
+    torch = _torch()
+    t = torch.empty((max_pos, head_dim // 2, 2), dtype=torch.float32, device=device)
+    check(wan_rope_freqs(head_dim, max_pos, theta, t.data_ptr(), _stream(stream)))
+    return t
+
+
+def workspace_bytes(dims: wan_dims, B: int) -> int:
+    n = wan_block_workspace_bytes(dims, B)
+    if n == 0 and B > 0:
+        raise WanError(WAN_EINVAL, last_error())
+    return n
+
+
+def alloc_workspace(dims: wan_dims, B: int, device="cuda"):
+    torch = _torch()
+    n = wan_block_workspace_bytes(dims, B)
+    if n == 0:
+        raise WanError(WAN_EINVAL, last_error())
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def workspace_view(ws, dims: wan_dims, B: int, which: int, shape, dtype):
+    """A tensor view of one workspace buffer (see WAN_WS_* in include/wan.h)."""
+    torch = _torch()
+    off = wan_block_workspace_offset(dims, B, which)
+    n = 1
+    for s in shape:
+        n *= s
+    es = torch.empty((), dtype=dtype).element_size()
+    return ws[off:off + n * es].view(dtype).view(*shape)
+
+
+def block_forward(dims: wan_dims, x, ctx, e0, weights, rope, workspace, ctx_lens=None,
+                  stream=None, cweights=None):
+    """One block in place on x ([B, L, dim] float32). ``weights`` is a dict of
+    device tensors (see WEIGHT_FIELDS) or a prebuilt wan_block_weights."""
+    B = x.shape[0]
+    cw = weights if isinstance(weights, wan_block_weights) else make_weights(weights)
+    check(wan_block_forward(dims, B, x.data_ptr(), _ptr(ctx), _ptr(ctx_lens), e0.data_ptr(), cw,
+                            rope.data_ptr(), rope.shape[0], workspace.data_ptr(),
+                            workspace.numel() * workspace.element_size(), _stream(stream)))
+    return x
+
+
+def attention(q, k, v, k_lens=None, scale=0.0, grid=None, rope=None, out=None, stream=None):
+    """q [B, Lq, n, d], k/v [B, Lk, n, d] (bf16 or f32). With ``grid`` the
+    3D RoPE is applied to q and k in place first."""
+    torch = _torch()
+    B, Lq, n, d = q.shape
+    Lk = k.shape[1]
+    o = torch.empty_like(q) if out is None else out
+    check(wan_attention(B, n, Lq, Lk, d, dtype_code(q), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                        o.data_ptr(), _ptr(k_lens), scale, grid, _ptr(rope),
+                        0 if rope is None else rope.shape[0], _stream(stream)))
+    return o
+
+
+def euler_cfg_step(x, v_cond, v_uncond, guide_scale, sigma, sigma_next, stream=None):
+    check(wan_euler_cfg_step(x.data_ptr(), v_cond.data_ptr(), _ptr(v_uncond), dtype_code(v_cond),
+                             x.numel(), guide_scale, sigma, sigma_next, _stream(stream)))
+    return x
+
+
+def device_status(stream=None) -> int:
+    return wan_device_status(_stream(stream))
