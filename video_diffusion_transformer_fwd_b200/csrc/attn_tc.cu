@@ -1,6 +1,336 @@
-// placeholder, replaced by the tcgen05 flash attention
+// Flash attention forward for sm_100a: bf16 q, k, v with head_dim 128,
+// non-causal, online softmax in fp32, tensor-core products accumulated in TMEM.
+// ("Wan2.2 code walkthrough" (newtid.com), self-attention snippet: global
+// window, key lengths; softmax(q k^T * scale) v.)
+//
+// One CTA = 2 query tiles of 128 rows of one (sequence, head):
+//   warps 0..3 / 4..7  softmax of query tile 0 / 1: thread = one query row;
+//               reads its row of S (128 keys, fp32) from TMEM, keeps a running
+//               max m (log2 domain) and sum l, writes P = exp2(S c - m) as bf16
+//               back into the first 64 columns of the same TMEM region, and
+//               rescales its O row in TMEM only when m grows by more than 8
+//               (P stays <= 2^8 otherwise, the final O / l is unchanged);
+//   warp 8      MMA issuer: S_i = Q_i K_j^T (A, B from shared memory), then
+//               O_i += P_i V_j (A = P from TMEM, B = V, MN-major, from
+//               shared memory);
+//   warp 9      TMA producer: Q tiles once, then K_j and V_j alternately into
+//               a 4-slot ring of 32 KB slots (128-byte swizzle).
+// TMEM: S_0 | S_1 | O_0 | O_1, 128 fp32 columns each (512 total).
+// Every wait is bounded (sm100::mbar_wait); keys at or beyond the sequence's
+// key length are masked; rows of a tile beyond Lq are computed but not stored.
 #include "common.cuh"
+#include "sm100.cuh"
+
 namespace wan {
-bool attention_tc_supported(const AttnArgs &) { return false; }
-int attention_tc(const AttnArgs &, cudaStream_t) { return set_error(WAN_EUNSUPPORTED, "attention_tc"); }
+
+namespace {
+using namespace sm100;
+
+constexpr int D = 128;                 // head_dim
+constexpr int TQ = 128;                // query rows per tile
+constexpr int TK = 128;                // keys per tile
+constexpr int NSLOT = 4;               // K/V ring slots
+constexpr int TILE_BYTES = 128 * D * 2;  // 32 KB: one Q, K or V tile (two 64-column boxes)
+constexpr int BOX_BYTES = TILE_BYTES / 2;
+constexpr int THREADS = 320;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t IDESC_S = idesc_bf16(TQ, TK, 0);
+constexpr uint32_t IDESC_O = idesc_bf16(TQ, D, 1);
+constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
+constexpr int SMEM_BYTES = 1024 + 2 * TILE_BYTES + NSLOT * TILE_BYTES + 256;
+
+struct FaParams {
+  int B, heads, Lq, Lk;
+  const int *k_lens;
+  float c;                    // scale * log2(e)
+  __nv_bfloat16 *o; int ldo;
+  int *watchdog;
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = smem;                               // 2 tiles
+  uint8_t *sKV = smem + 2 * TILE_BYTES;             // NSLOT tiles
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + NSLOT * TILE_BYTES);
+  uint64_t *q_full = bars;
+  uint64_t *kv_full = bars + 1;
+  uint64_t *kv_empty = bars + 1 + NSLOT;
+  uint64_t *s_full = bars + 1 + 2 * NSLOT;
+  uint64_t *p_ready = s_full + 2;
+  uint64_t *pv_done = p_ready + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pv_done + 2);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int q0 = blockIdx.x * 2 * TQ;
+  int kl = p.Lk;
+  if (p.k_lens) kl = min(max(p.k_lens[b], 0), p.Lk);
+  const int nkt = (kl + TK - 1) / TK;
+
+  // A CTA that starts after another one gave up a wait skips its work, so a
+  // failed launch ends within a few waits instead of one per CTA.
+  if (threadIdx.x == 0) *abort_flag = (p.watchdog && *reinterpret_cast<volatile int *>(p.watchdog)) ? 1 : 0;
+  __syncthreads();
+  if (*abort_flag) return;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(smem_u32(&kv_full[s]), 1);
+      mbar_init(smem_u32(&kv_empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&p_ready[i]), 4);
+      mbar_init(smem_u32(&pv_done[i]), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0 && nkt > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const uint32_t qb = smem_u32(q_full);
+      mbar_arrive_expect_tx(qb, 2 * TILE_BYTES);
+      for (int i = 0; i < 2; ++i)
+        for (int half = 0; half < 2; ++half)
+          tma_load_3d(smem_u32(sQ + i * TILE_BYTES + half * BOX_BYTES), &tmQ, h * D + half * 64,
+                      q0 + i * TQ, b, qb);
+      int slot = 0;
+      uint32_t phase = 0;
+      int fills[NSLOT] = {0, 0, 0, 0};
+      bool ok = true;
+      for (int j = 0; j < nkt && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv) {
+          if (!mbar_wait(smem_u32(&kv_empty[slot]), phase ^ 1, abort_flag, p.watchdog, 0x201)) { ok = false; break; }
+          const uint32_t fb = smem_u32(&kv_full[slot]);
+          mbar_arrive_expect_tx(fb, TILE_BYTES);
+          const CUtensorMap *tm = kv == 0 ? &tmK : &tmV;
+          for (int half = 0; half < 2; ++half)
+            tma_load_3d(smem_u32(sKV + slot * TILE_BYTES + half * BOX_BYTES), tm, h * D + half * 64,
+                        j * TK, b, fb);
+          ++fills[slot];
+          if (++slot == NSLOT) { slot = 0; phase ^= 1; }
+        }
+      }
+      int never = 0;
+      mbar_wait(qb, 0, &never, p.watchdog, 0x202);
+      for (int s = 0; s < NSLOT; ++s)
+        if (fills[s] > 0) mbar_wait(smem_u32(&kv_full[s]), (fills[s] - 1) & 1, &never, p.watchdog, 0x203);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0 && nkt > 0) {
+      bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.watchdog, 0x211);
+      int slot = 0;
+      uint32_t phase = 0;
+      for (int j = 0; j < nkt && ok; ++j) {
+        // S_i = Q_i K_j^T
+        if (!mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x212)) break;
+        const uint32_t kbase = smem_u32(sKV + slot * TILE_BYTES);
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (j > 0 && !mbar_wait(smem_u32(&pv_done[i]), (j - 1) & 1, abort_flag, p.watchdog, 0x213)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qbase = smem_u32(sQ + i * TILE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
+            mma_ss(tmem + i * TK, desc_kmajor_sw128(qbase + off), desc_kmajor_sw128(kbase + off), IDESC_S, kk > 0);
+          }
+          tc_commit(smem_u32(&s_full[i]));
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&kv_empty[slot]));
+        if (++slot == NSLOT) { slot = 0; phase ^= 1; }
+        // O_i += P_i V_j
+        if (!mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x214)) break;
+        const uint32_t vbase = smem_u32(sKV + slot * TILE_BYTES);
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (!mbar_wait(smem_u32(&p_ready[i]), j & 1, abort_flag, p.watchdog, 0x215)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < TK / 16; ++kk)
+            mma_ts(tmem + 2 * TK + i * D, tmem + i * TK + kk * 8,
+                   desc_mnmajor_sw128(vbase + kk * 16 * 128, BOX_BYTES, 1024), IDESC_O, (j > 0 || kk > 0));
+          tc_commit(smem_u32(&pv_done[i]));
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&kv_empty[slot]));
+        if (++slot == NSLOT) { slot = 0; phase ^= 1; }
+      }
+    }
+  } else {
+    // ------------------------------------------------ softmax (warps 0..7)
+    const int i = warp >> 2;                       // query tile
+    const int qw = warp & 3;                       // TMEM lane quarter
+    const int row = q0 + i * TQ + qw * 32 + lane;  // query row in the sequence
+    const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
+    const uint32_t s_addr = tmem + lane_off + i * TK;
+    const uint32_t o_addr = tmem + lane_off + 2 * TK + i * D;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkt; ++j) {
+      if (!mbar_wait(smem_u32(&s_full[i]), j & 1, abort_flag, p.watchdog, 0x221)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
+      tmem_ld_wait();
+      const int kvalid = kl - j * TK;              // keys of this tile that are valid
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 128; ++k) {
+        float x = __uint_as_float(s[k]) * p.c;
+        if (k >= kvalid) x = -INFINITY;
+        s[k] = __float_as_uint(x);
+        tmax = fmaxf(tmax, x);
+      }
+      // running max with conditional rescaling of l and O; the TMEM accesses
+      // are warp-collective, so a warp rescales when any of its rows must
+      const bool need = (tmax > m + RESCALE_THRESHOLD) || (m == -INFINITY);
+      const float mnew = need ? tmax : m;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        const float alpha = need ? ex2(m - mnew) : 1.0f;
+        l *= alpha;
+        if (!mbar_wait(smem_u32(&pv_done[i]), (j - 1) & 1, abort_flag, p.watchdog, 0x222)) ok = false;
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + c * 32, o);
+          tmem_ld_wait();
+          uint32_t a[16], bq[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            a[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            bq[e] = __float_as_uint(__uint_as_float(o[16 + e]) * alpha);
+          }
+          tmem_st16(o_addr + c * 32, a);
+          tmem_st16(o_addr + c * 32 + 16, bq);
+        }
+        tmem_st_wait();
+      }
+      m = mnew;
+      // P = exp2(x - m) as bf16 pairs into the first 64 columns of S_i
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2(__uint_as_float(s[c * 32 + 2 * e]) - m);
+          const float p1 = ex2(__uint_as_float(s[c * 32 + 2 * e + 1]) - m);
+          rs += p0 + p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        tmem_st16(s_addr + c * 16, pk);
+      }
+      l += rs;
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&p_ready[i]));
+      if (!ok) break;
+    }
+    // epilogue: O / l -> bf16
+    if (ok && nkt > 0) {
+      ok = mbar_wait(smem_u32(&pv_done[i]), (nkt - 1) & 1, abort_flag, p.watchdog, 0x223);
+      tc_fence_after();
+    }
+    const float inv = (l > 0.f) ? 1.0f / l : 0.f;
+    __nv_bfloat16 *orow = p.o + (size_t)(b * p.Lq + (row < p.Lq ? row : 0)) * p.ldo + h * D;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t o[32];
+      if (nkt > 0) {
+        tmem_ld32(o_addr + c * 32, o);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (row < p.Lq && ok) {
+        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint4 u;
+          u.x = pack_bf16(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
+          u.y = pack_bf16(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
+          u.z = pack_bf16(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
+          u.w = pack_bf16(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
+          dst[e] = u;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 8) tmem_dealloc(tmem, TMEM_COLS);
+}
+}  // namespace
+
+bool attention_tc_supported(const AttnArgs &a) {
+  if (a.d != D || a.B < 1 || a.Lq < 1 || a.Lk < 0) return false;
+  if (a.ldq % 8 || a.ldk % 8 || a.ldv % 8 || a.ldo % 8) return false;
+  if (!aligned16(a.q) || !aligned16(a.k) || !aligned16(a.v) || !aligned16(a.o)) return false;
+  if (a.heads > 65535 || a.B > 65535) return false;
+  return true;
+}
+
+int attention_tc(const AttnArgs &a, cudaStream_t s) {
+  if (!attention_tc_supported(a)) return set_error(WAN_EUNSUPPORTED, "attention_tc");
+  const int Lk = a.Lk > 0 ? a.Lk : 1;
+  CUtensorMap tq, tk, tv;
+  const uint64_t inner = (uint64_t)a.heads * D;
+  int rc = encode_tmap_3d_bf16(&tq, a.q, inner, a.Lq, a.B, (uint64_t)a.ldq * 2, (uint64_t)a.Lq * a.ldq * 2, 64, TQ);
+  if (rc) return rc;
+  if ((rc = encode_tmap_3d_bf16(&tk, a.k, inner, Lk, a.B, (uint64_t)a.ldk * 2, (uint64_t)a.Lk * a.ldk * 2 + (a.Lk ? 0 : 16), 64, TK))) return rc;
+  if ((rc = encode_tmap_3d_bf16(&tv, a.v, inner, Lk, a.B, (uint64_t)a.ldv * 2, (uint64_t)a.Lk * a.ldv * 2 + (a.Lk ? 0 : 16), 64, TK))) return rc;
+  static bool attr_set = false;
+  if (!attr_set) {
+    WAN_TRY_CUDA(cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
+                 "attention_tc smem attribute");
+    attr_set = true;
+  }
+  FaParams p = {};
+  p.B = a.B; p.heads = a.heads; p.Lq = a.Lq; p.Lk = a.Lk; p.k_lens = a.k_lens;
+  p.c = a.scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16 *>(a.o); p.ldo = a.ldo;
+  p.watchdog = watchdog_ptr();
+  dim3 grid((a.Lq + 2 * TQ - 1) / (2 * TQ), a.heads, a.B);
+  attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tq, tk, tv, p);
+  WAN_CHECK_LAUNCH("attention_tc");
+  return WAN_OK;
+}
+
+}  // namespace wan

@@ -58,7 +58,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // WAIT_LIMIT_NS or when another thread of the CTA has raised `*abort`; on
 // giving up it records `code` in the library's watchdog word and raises
 // `*abort`, and returns false. Never traps.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
+static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                        int *watchdog, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
