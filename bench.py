@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark of the Wan DiT hot path on B200: one A14B-shaped denoising step
+per bench step (40 WanAttentionBlocks, dim 5120, 40 heads, ffn 13824, on the
+CFG pair -- cond and uncond batched as B = 2 -- over L = 32760 tokens, then
+the CFG-Euler update x += (sigma' - sigma) v with guidance 5, sigma 0.9 ->
+0.875), all through the C ABI of libwan.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). The metric is the DiT block forward time:
+`value` = device time of the timed steps / (steps x blocks x 2 sequences x
+N ranks), i.e. ms per block forward over one 32760-token sequence for the
+whole job (lower is better); attention and GEMM TFLOP/s come from CUDA
+events recorded around every kernel launch inside the timed region.
+Multi-GPU runs are independent replicas (each rank its own step; weak
+scaling), timed as the max over ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DiT block fwd ms & attention TFLOP/s (bf16, 32760 tok) vs tensor peak"
+UNIT = "ms per block forward (one 32760-token sequence)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic per launch of the dominant kernel, from an ncu capture of the
+# same kernel source (sha256 prefix below); reported as null once the source
+# has changed since the capture.
+TRAFFIC = {}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="a14b-step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(name):
+    p = os.path.join(ROOT, "video_diffusion_transformer_fwd_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, indices):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", ",".join(str(i) for i in indices)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], [], set(), []
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- CPU oracle sample
+class OracleSample:
+    """Times the fp64 oracle (as it stands) on a bounded sample of one block
+    forward of the workload and expresses it per block forward of one
+    sequence: LayerNorm + K/V projection on r_kv rows (scaled by L / r_kv),
+    and the rest of the block for r_q and 2 r_q query rows attending over
+    all L keys (the difference gives the per-row cost, the remainder the
+    fixed per-call cost of the text K/V projection). Inputs are drawn once
+    by the seeded generators; only the oracle calls are timed."""
+
+    def __init__(self, cfg, seed=0, r_kv=512, r_q=2):
+        import numpy as np
+
+        from video_diffusion_transformer_fwd_b200 import synth
+        self.cfg, self.r_kv, self.r_q = cfg, r_kv, r_q
+        w = synth.block_weights(cfg.dim, cfg.ffn_dim, cfg.dtype, "cpu", seed)
+        self.w64 = {k: synth.to_numpy64(v) for k, v in w.items()}
+        acts = synth.block_activations(1, r_kv, cfg.dim, cfg.text_len, cfg.dtype, "cpu", seed + 100)
+        self.x = synth.to_numpy64(acts["x"])
+        self.ctx = synth.to_numpy64(acts["ctx"])
+        self.e0 = synth.to_numpy64(acts["e0"])
+        reps = (cfg.L + r_kv - 1) // r_kv
+        self.xq = np.ascontiguousarray(np.tile(self.x, (1, reps, 1))[:, :cfg.L])
+        self.reps = reps
+
+    def run(self):
+        import numpy as np
+
+        from oracle import wan_oracle as O
+        cfg, r_kv, r_q = self.cfg, self.r_kv, self.r_q
+        t0 = time.perf_counter()
+        k, v = O.self_attn_kv(self.x, self.e0, self.w64, cfg.heads, (1, 1, r_kv), cfg.eps, cfg.theta)
+        t_kv = time.perf_counter() - t0
+        # full-length keys/values (rows repeated: the attention cost depends only on L)
+        kf = np.tile(k, (1, self.reps, 1, 1))[:, :cfg.L]
+        vf = np.tile(v, (1, self.reps, 1, 1))[:, :cfg.L]
+        grid = (cfg.F, cfg.H, cfg.W)
+        times = []
+        for r in (r_q, 2 * r_q):
+            t0 = time.perf_counter()
+            O.block_forward_rows(self.xq, self.ctx, None, self.e0, self.w64, cfg.heads, grid, cfg.eps,
+                                 np.arange(r), theta=cfg.theta, kv=(kf, vf))
+            times.append(time.perf_counter() - t0)
+        per_row = max((times[1] - times[0]) / r_q, 0.0)
+        fixed = max(times[0] - per_row * r_q, 0.0)
+        est = t_kv * cfg.L / r_kv + fixed + per_row * cfg.L
+        detail = (f"fp64 oracle on one block forward of the workload's block shape (one sequence): "
+                  f"LN + K/V projection timed on {r_kv} rows (scaled x{cfg.L / r_kv:.1f}); the rest "
+                  f"of the block timed for {r_q} and {2 * r_q} query rows attending over all {cfg.L} "
+                  f"keys (per-row cost x{cfg.L}, plus the per-call text K/V projection); "
+                  f"{t_kv + sum(times):.1f} s of CPU time sampled")
+        return est * 1e3, detail
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return sum(i.get("num_threads", 0) for i in info if i.get("user_api") == "blas") or None
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from video_diffusion_transformer_fwd_b200 import configs
+    cfg = configs.get(args.config)
+    sample = OracleSample(cfg, seed=0)
+    vals = []
+    detail = ""
+    for i in range(args.warmup + args.steps):
+        ms, detail = sample.run()
+        if i >= args.warmup:
+            vals.append(ms)
+    value = statistics.mean(vals)
+    cores = cpu_cores()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": value * cfg.blocks * 2, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": workload_config(cfg, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "blas_threads": blas_threads(),
+                         "kind": "oracle", "sample": detail},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg, world):
+    return {
+        "workload": (f"{cfg.name}: {cfg.blocks} WanAttentionBlocks dim {cfg.dim}, {cfg.heads} heads "
+                     f"(head_dim {cfg.head_dim}), ffn {cfg.ffn_dim}, grid {cfg.F}x{cfg.H}x{cfg.W} "
+                     f"(L={cfg.L}), text {cfg.text_len}, cond+uncond batched (B=2), CFG "
+                     f"{cfg.guide_scale}, Euler sigma {cfg.sigma}->{cfg.sigma_next}"),
+        "seq_len": cfg.L, "batch_per_gpu": 2, "blocks": cfg.blocks, "global_batch": 2 * world,
+        "parallelism": "replicas" if world > 1 else "single",
+        "l2": "inputs larger than L2 (28 GB of block weights and a 671 MB token state per step)",
+        "weights": "random N(0,0.02), synthetic x/ctx N(0,1)",
+    }
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from video_diffusion_transformer_fwd_b200 import configs, wan
+    from video_diffusion_transformer_fwd_b200.step import DenoiseStep
+
+    torch.cuda.set_device(local_rank)
+    dev = f"cuda:{local_rank}"
+    cfg = configs.get(args.config)
+    st = DenoiseStep(cfg, seed=1000 * rank, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        st.step()
+    torch.cuda.synchronize()
+    if wan.device_status() != wan.WAN_OK:
+        raise RuntimeError("warm-up: " + wan.last_error())
+
+    clocks = ClockSampler(list(range(world)) if rank == 0 else [local_rank]) if rank == 0 else None
+    wan.check(wan.wan_profile_enable(1))
+    barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wall0 = time.perf_counter()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        st.step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - wall0
+    ms_total = t_start.elapsed_time(t_end)
+    prof = wan.profile_read()
+    wan.check(wan.wan_profile_enable(0))
+    clock_info = clocks.stop() if clocks else None
+    if wan.device_status() != wan.WAN_OK:
+        raise RuntimeError("timed region: " + wan.last_error())
+
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # end to end: host (pinned) inputs in, result out, every step
+    e2e = None
+    if not args.no_e2e:
+        x_h = torch.empty(st.x.shape, dtype=st.x.dtype, pin_memory=True)
+        x_h.copy_(st.x)
+        ctx_h = torch.empty(st.ctx.shape, dtype=st.ctx.dtype, pin_memory=True)
+        ctx_h.copy_(st.ctx)
+        e0_h = torch.empty(st.e0.shape, dtype=st.e0.dtype, pin_memory=True)
+        e0_h.copy_(st.e0)
+        out_h = torch.empty_like(x_h, pin_memory=True)
+        h2d = x_h.numel() * x_h.element_size() + ctx_h.numel() * ctx_h.element_size() + \
+            e0_h.numel() * e0_h.element_size()
+        d2h = out_h.numel() * out_h.element_size()
+        barrier()
+        torch.cuda.synchronize()
+        e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e_start.record(stream)
+        for _ in range(args.steps):
+            st.x.copy_(x_h, non_blocking=True)
+            st.ctx.copy_(ctx_h, non_blocking=True)
+            st.e0.copy_(e0_h, non_blocking=True)
+            st.step()
+            out_h.copy_(st.x, non_blocking=True)
+        e_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        te = torch.tensor([e_start.elapsed_time(e_end)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        units = args.steps * cfg.blocks * 2 * world
+        e2e = {"value": float(te.item()) / units, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+
+    if rank != 0:
+        return
+    units = args.steps * cfg.blocks * 2 * world
+    value = ms_max / units
+    peaks, peak_src = read_peaks()
+    blocks_run = args.steps * cfg.blocks
+    import dataclasses
+    c2 = dataclasses.replace(cfg, batch=2)
+    attn_n, attn_ms = prof["attn_self"]
+    gemm_n, gemm_ms = prof["gemm_tc"]
+    attn_flops_launch = c2.self_attn_flops()
+    attn_tflops = attn_flops_launch * attn_n / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else None
+    gemm_tflops = c2.gemm_flops() * blocks_run / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    # dominant kernel class by device time
+    dom = max(prof.items(), key=lambda kv: kv[1][1])[0]
+    peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    roofline = None
+    if dom == "attn_self" and attn_n:
+        avg_ms = attn_ms / attn_n
+        tr = TRAFFIC.get("attn_self")
+        traffic = None
+        if tr and tr.get("source_sha") == source_hash("attn_tc.cu"):
+            traffic = tr["bytes_per_launch"]
+        roofline = {"kernel": "attn_tc (self-attention, B=2, L=32760, 40 heads, d=128)",
+                    "bound": "tensor", "achieved": attn_flops_launch / (avg_ms * 1e-3) / 1e12,
+                    "peak": peak_sust, "unit": "TFLOP/s",
+                    "frac": attn_flops_launch / (avg_ms * 1e-3) / 1e12 / peak_sust,
+                    "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                    "traffic": traffic, "avg_launch_ms": avg_ms,
+                    "algorithmic_flops_per_launch": attn_flops_launch}
+    elif dom == "gemm_tc" and gemm_n:
+        roofline = {"kernel": "gemm_tc (all block GEMMs)", "bound": "tensor", "achieved": gemm_tflops,
+                    "peak": peak_sust, "unit": "TFLOP/s", "frac": gemm_tflops / peak_sust,
+                    "peak_source": f"{peak_src} bf16 sustained", "traffic": None}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "impl": "ours",
+        "config": workload_config(cfg, world),
+        "attention_tflops": attn_tflops, "gemm_tflops": gemm_tflops,
+        "attention_frac_of_2250": None if attn_tflops is None else attn_tflops / 2250.0,
+        "gemm_frac_of_2250": None if gemm_tflops is None else gemm_tflops / 2250.0,
+        "kernel_ms_per_step": {k: v[1] / args.steps for k, v in prof.items() if v[0]},
+        "gpu_launches": sum(v[0] for v in prof.values()),
+        "roofline": roofline,
+        "clocks": clock_info,
+        "wall_s_timed": wall,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        ms, detail = OracleSample(cfg, seed=0).run()
+        line["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": cpu_cores(),
+                                "blas_threads": blas_threads(), "kind": "oracle", "sample": detail}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device(f"cuda:{local_rank}"))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -186,6 +186,27 @@ int wan_euler_cfg_step(float *x, const void *v_cond, const void *v_uncond,
  * outputs are then invalid), or WAN_ECUDA if the stream holds a CUDA error. */
 int wan_device_status(wan_stream_t stream);
 
+/* Launch instrumentation. While enabled, every kernel the library launches is
+ * bracketed by two CUDA events recorded on its stream (a few microseconds of
+ * host overhead per launch). wan_profile_enable(on) also clears the record;
+ * wan_profile_read waits for the recorded events and returns, for one kernel
+ * class, the number of launches and their summed device time in ms. Events
+ * are created on first use and reused; at most 65536 launches are recorded.
+ * Not thread-safe against concurrent enable/read. */
+#define WAN_K_GEMM_TC      0  /* tensor-core GEMM (any epilogue)              */
+#define WAN_K_GEMM_SIMT    1  /* CUDA-core GEMM                               */
+#define WAN_K_ATTN_SELF    2  /* tensor-core attention, self (block)          */
+#define WAN_K_ATTN_CROSS   3  /* tensor-core attention, cross (block)         */
+#define WAN_K_ATTN_SIMT    4  /* CUDA-core attention                          */
+#define WAN_K_LAYERNORM    5  /* LayerNorm + modulation / affine              */
+#define WAN_K_QKNORM_ROPE  6  /* q/k RMSNorm and/or 3D RoPE                   */
+#define WAN_K_EULER        7  /* CFG + Euler update                           */
+#define WAN_K_MISC         8  /* modulation combine, RoPE table               */
+#define WAN_K_ATTN_TC      9  /* tensor-core attention via wan_attention      */
+#define WAN_K_COUNT       10
+int wan_profile_enable(int on);
+int wan_profile_read(int kernel_class, int *launches, double *total_ms);
+
 #ifdef __cplusplus
 }
 #endif

@@ -48,13 +48,14 @@ int *watchdog_ptr() {
 
 // ---------------------------------------------------------------- dispatch
 static int run_gemm(const GemmArgs &g, int dtype, cudaStream_t s) {
-  if (dtype == WAN_BF16 && gemm_tc_supported(g)) return gemm_tc(g, s);
-  return gemm_simt(g, dtype, s);
+  if (dtype == WAN_BF16 && gemm_tc_supported(g)) return WAN_PROF(WAN_K_GEMM_TC, s, gemm_tc(g, s));
+  return WAN_PROF(WAN_K_GEMM_SIMT, s, gemm_simt(g, dtype, s));
 }
 
-static int run_attention(const AttnArgs &a, int dtype, cudaStream_t s) {
-  if (dtype == WAN_BF16 && attention_tc_supported(a)) return attention_tc(a, s);
-  return attention_simt(a, dtype, s);
+// cls: profiling class used when the tensor-core kernel runs
+static int run_attention(const AttnArgs &a, int dtype, cudaStream_t s, int cls) {
+  if (dtype == WAN_BF16 && attention_tc_supported(a)) return WAN_PROF(cls, s, attention_tc(a, s));
+  return WAN_PROF(WAN_K_ATTN_SIMT, s, attention_simt(a, dtype, s));
 }
 
 // ---------------------------------------------------------------- workspace
@@ -125,7 +126,7 @@ int wan_rope_freqs(int head_dim, int max_pos, double theta, float *table, wan_st
   if (!(theta > 0.0)) return set_error(WAN_EINVAL, "theta must be > 0");
   if (!table) return set_error(WAN_EINVAL, "table is NULL");
   if (!aligned16(table)) return set_error(WAN_EALIGN, "table not 16-byte aligned");
-  return launch_rope_table(head_dim, max_pos, theta, table, (cudaStream_t)stream);
+  return WAN_PROF(WAN_K_MISC, (cudaStream_t)stream, launch_rope_table(head_dim, max_pos, theta, table, (cudaStream_t)stream));
 }
 
 size_t wan_block_workspace_bytes(const wan_dims *dims, int B) {
@@ -180,10 +181,10 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
   const int BL = B * L;
 
   // m = modulation + e0  (shift, scale, gate, shift2, scale2, gate2)
-  if ((rc = launch_mod_combine(w->modulation, e0, mod, B, D, s))) return rc;
+  if ((rc = WAN_PROF(WAN_K_MISC, s, launch_mod_combine(w->modulation, e0, mod, B, D, s)))) return rc;
 
   // ---- self-attention branch: x += m2 * Wo . Attn(RoPE(RMSNorm(q,k)), v)
-  if ((rc = launch_layernorm_mod(x, act, dt, BL, D, L, mod, 0, 1, nullptr, nullptr, d.eps, s))) return rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, L, mod, 0, 1, nullptr, nullptr, d.eps, s)))) return rc;
   {
     GemmArgs g = {};
     g.M = BL; g.N = 3 * D; g.K = D; g.A = act; g.lda = D;
@@ -192,14 +193,14 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
     g.segN = D; g.nseg = 3; g.epi = EPI_STORE; g.C = qkv; g.ldc = 3 * D;
     if ((rc = run_gemm(g, dt, s))) return rc;
   }
-  if ((rc = launch_rmsnorm_rope(qkv, dt, BL, 3 * D, D, hd, w->gq, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s))) return rc;
-  if ((rc = launch_rmsnorm_rope(qkv + D * es, dt, BL, 3 * D, D, hd, w->gk, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s))) return rc;
+  if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qkv, dt, BL, 3 * D, D, hd, w->gq, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s)))) return rc;
+  if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qkv + D * es, dt, BL, 3 * D, D, hd, w->gk, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s)))) return rc;
   {
     AttnArgs a = {};
     a.B = B; a.heads = d.heads; a.Lq = L; a.Lk = L; a.d = hd;
     a.q = qkv; a.ldq = 3 * D; a.k = qkv + D * es; a.ldk = 3 * D; a.v = qkv + 2 * D * es; a.ldv = 3 * D;
     a.o = o; a.ldo = D; a.k_lens = nullptr; a.scale = 1.0f / sqrtf((float)hd);
-    if ((rc = run_attention(a, dt, s))) return rc;
+    if ((rc = run_attention(a, dt, s, WAN_K_ATTN_SELF))) return rc;
   }
   {
     GemmArgs g = {};
@@ -210,7 +211,7 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
   }
 
   // ---- cross-attention branch (ungated): x += Wco . Attn(q(norm3 x), k(ctx), v(ctx))
-  if ((rc = launch_layernorm_mod(x, act, dt, BL, D, L, nullptr, 0, 0, w->g3, w->b3, d.eps, s))) return rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, L, nullptr, 0, 0, w->g3, w->b3, d.eps, s)))) return rc;
   {
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = D; g.A = act; g.lda = D;
@@ -218,21 +219,21 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
     g.epi = EPI_STORE; g.C = qc; g.ldc = D;
     if ((rc = run_gemm(g, dt, s))) return rc;
   }
-  if ((rc = launch_rmsnorm_rope(qc, dt, BL, D, D, hd, w->cgq, d.eps, nullptr, 0, 1, 1, 1, s))) return rc;
+  if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qc, dt, BL, D, D, hd, w->cgq, d.eps, nullptr, 0, 1, 1, 1, s)))) return rc;
   if (T > 0) {
     GemmArgs g = {};
     g.M = B * T; g.N = 2 * D; g.K = D; g.A = ctx; g.lda = D;
     g.Bseg[0] = w->cwk; g.Bseg[1] = w->cwv; g.bias[0] = w->cbk; g.bias[1] = w->cbv;
     g.segN = D; g.nseg = 2; g.epi = EPI_STORE; g.C = kvc; g.ldc = 2 * D;
     if ((rc = run_gemm(g, dt, s))) return rc;
-    if ((rc = launch_rmsnorm_rope(kvc, dt, B * T, 2 * D, D, hd, w->cgk, d.eps, nullptr, 0, 1, 1, 1, s))) return rc;
+    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(kvc, dt, B * T, 2 * D, D, hd, w->cgk, d.eps, nullptr, 0, 1, 1, 1, s)))) return rc;
   }
   {
     AttnArgs a = {};
     a.B = B; a.heads = d.heads; a.Lq = L; a.Lk = T; a.d = hd;
     a.q = qc; a.ldq = D; a.k = kvc; a.ldk = 2 * D; a.v = kvc + D * es; a.ldv = 2 * D;
     a.o = oc; a.ldo = D; a.k_lens = ctx_lens; a.scale = 1.0f / sqrtf((float)hd);
-    if ((rc = run_attention(a, dt, s))) return rc;
+    if ((rc = run_attention(a, dt, s, WAN_K_ATTN_CROSS))) return rc;
   }
   {
     GemmArgs g = {};
@@ -243,7 +244,7 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
   }
 
   // ---- FFN branch: x += m5 * W2 . gelu_tanh(W1 . (LN(x)(1 + m4) + m3))
-  if ((rc = launch_layernorm_mod(x, act, dt, BL, D, L, mod, 3, 4, nullptr, nullptr, d.eps, s))) return rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, L, mod, 3, 4, nullptr, nullptr, d.eps, s)))) return rc;
   {
     GemmArgs g = {};
     g.M = BL; g.N = Fh; g.K = D; g.A = act; g.lda = D;
@@ -298,14 +299,14 @@ int wan_attention(int B, int heads, int Lq, int Lk, int head_dim, int dtype, voi
     const int gmax = F > H ? (F > W ? F : W) : (H > W ? H : W);
     if (!rope || rope_max_pos < gmax) return set_error(WAN_EINVAL, "rope table missing or too short");
     if (!aligned16(rope)) return set_error(WAN_EALIGN, "rope not 16-byte aligned");
-    if ((rc = launch_rope_only(q, dtype, B * Lq, D, D, head_dim, rope, rope_max_pos, F, H, W, s))) return rc;
-    if ((rc = launch_rope_only(k, dtype, B * Lk, D, D, head_dim, rope, rope_max_pos, F, H, W, s))) return rc;
+    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rope_only(q, dtype, B * Lq, D, D, head_dim, rope, rope_max_pos, F, H, W, s)))) return rc;
+    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rope_only(k, dtype, B * Lk, D, D, head_dim, rope, rope_max_pos, F, H, W, s)))) return rc;
   }
   AttnArgs a = {};
   a.B = B; a.heads = heads; a.Lq = Lq; a.Lk = Lk; a.d = head_dim;
   a.q = q; a.ldq = D; a.k = k; a.ldk = D; a.v = v; a.ldv = D; a.o = o; a.ldo = D;
   a.k_lens = k_lens; a.scale = scale != 0.f ? scale : 1.0f / sqrtf((float)head_dim);
-  return run_attention(a, dtype, s);
+  return run_attention(a, dtype, s, WAN_K_ATTN_TC);
 }
 
 int wan_euler_cfg_step(float *x, const void *v_cond, const void *v_uncond, int v_dtype, size_t n,
@@ -316,8 +317,9 @@ int wan_euler_cfg_step(float *x, const void *v_cond, const void *v_uncond, int v
   if (v_dtype != WAN_F32 && v_dtype != WAN_BF16) return set_error(WAN_EUNSUPPORTED, "v_dtype %d", v_dtype);
   if (!aligned16(x) || !aligned16(v_cond) || (v_uncond && !aligned16(v_uncond)))
     return set_error(WAN_EALIGN, "pointer not 16-byte aligned");
-  return launch_euler_cfg(x, v_cond, v_uncond, v_dtype, n, guide_scale, sigma_next - sigma,
-                          (cudaStream_t)stream);
+  cudaStream_t s = (cudaStream_t)stream;
+  return WAN_PROF(WAN_K_EULER, s, launch_euler_cfg(x, v_cond, v_uncond, v_dtype, n, guide_scale,
+                                                    sigma_next - sigma, s));
 }
 
 int wan_device_status(wan_stream_t stream) {

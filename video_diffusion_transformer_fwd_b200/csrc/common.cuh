@@ -151,4 +151,13 @@ int launch_rope_table(int head_dim, int max_pos, double theta, float *table, cud
 int launch_euler_cfg(float *x, const void *vc, const void *vu, int vdt, size_t n, float scale,
                      float dt, cudaStream_t s);
 
+// Brackets one kernel launch with profiling events when profiling is on.
+struct ProfScope {
+  int idx;
+  cudaStream_t stream;
+  ProfScope(int cls, cudaStream_t s);
+  ~ProfScope();
+};
+#define WAN_PROF(cls, s, expr) ([&]() { ::wan::ProfScope ps_((cls), (s)); return (expr); }())
+
 }  // namespace wan

@@ -18,6 +18,11 @@ WAN_OK, WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED, WAN_ECUDA, WAN_ETIMEOUT = 0, -
 WAN_F32, WAN_BF16 = 0, 1
 (WAN_WS_ACT, WAN_WS_QKV, WAN_WS_O, WAN_WS_QC, WAN_WS_KVC, WAN_WS_OC, WAN_WS_H, WAN_WS_MOD,
  WAN_WS_STATS) = range(9)
+(WAN_K_GEMM_TC, WAN_K_GEMM_SIMT, WAN_K_ATTN_SELF, WAN_K_ATTN_CROSS, WAN_K_ATTN_SIMT, WAN_K_LAYERNORM,
+ WAN_K_QKNORM_ROPE, WAN_K_EULER, WAN_K_MISC, WAN_K_ATTN_TC) = range(10)
+WAN_K_COUNT = 10
+KERNEL_CLASS_NAMES = ("gemm_tc", "gemm_simt", "attn_self", "attn_cross", "attn_simt", "layernorm",
+                      "qknorm_rope", "euler_cfg", "misc", "attn_tc")
 STATUS_NAMES = {0: "WAN_OK", -1: "WAN_EINVAL", -2: "WAN_EALIGN", -3: "WAN_EUNSUPPORTED",
                 -4: "WAN_ECUDA", -5: "WAN_ETIMEOUT"}
 
@@ -57,6 +62,8 @@ _SIGS = {
     "wan_euler_cfg_step": (_c_int, [_vp, _vp, _vp, _c_int, _sz, ctypes.c_float, ctypes.c_float,
                                     ctypes.c_float, _vp]),
     "wan_device_status": (_c_int, [_vp]),
+    "wan_profile_enable": (_c_int, [_c_int]),
+    "wan_profile_read": (_c_int, [_c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]),
 }
 
 _lib = None
@@ -126,6 +133,25 @@ def wan_euler_cfg_step(x, v_cond, v_uncond, v_dtype, n, guide_scale, sigma, sigm
 
 def wan_device_status(stream):
     return load().wan_device_status(stream)
+
+
+def wan_profile_enable(on):
+    return load().wan_profile_enable(on)
+
+
+def wan_profile_read(kernel_class, launches, total_ms):
+    return load().wan_profile_read(kernel_class, launches, total_ms)
+
+
+def profile_read():
+    """{class name: (launches, total device ms)} of the current record."""
+    out = {}
+    for c in range(WAN_K_COUNT):
+        n = ctypes.c_int(0)
+        ms = ctypes.c_double(0.0)
+        check(wan_profile_read(c, ctypes.byref(n), ctypes.byref(ms)))
+        out[KERNEL_CLASS_NAMES[c]] = (n.value, ms.value)
+    return out
 
 
 # ---------------------------------------------------------------- torch helpers
