@@ -149,6 +149,30 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx,
                       int rope_max_pos, void *workspace, size_t ws_bytes,
                       wan_stream_t stream);
 
+/* wan_block_forward_noalloc -- wan_block_forward without a caller-supplied
+ * workspace, for callers that cannot allocate device memory: a plug-in that
+ * only receives buffers from a host framework which owns the GPU's memory
+ * pool, a serving process whose memory budget is fixed up front, or a
+ * latency-critical loop where an allocation (which can synchronise the
+ * device) is not allowed. The pages have no counterpart to this entry point;
+ * it exists only for such callers.
+ *   Same arguments and results as wan_block_forward, minus workspace and
+ *   ws_bytes. The workspace is a built-in device array of
+ *   WAN_NOALLOC_WORKSPACE_BYTES bytes that every GPU loading the library
+ *   holds until the process exits; the entry point itself allocates nothing.
+ *   Problems with wan_block_workspace_bytes(dims, B) above that size are
+ *   rejected (WAN_EINVAL, message names both sizes).
+ *   The array's device address is looked up on the first call made with a
+ *   given device current: make that first call before any stream capture.
+ *   All calls on a device share the array and it keeps the previous call's
+ *   contents (the block writes every byte it reads, so no clearing is
+ *   needed); calls that may overlap on the GPU race on it. */
+#define WAN_NOALLOC_WORKSPACE_BYTES (16u << 20)
+int wan_block_forward_noalloc(const wan_dims *dims, int B, float *x, const void *ctx,
+                              const int *ctx_lens, const float *e0,
+                              const wan_block_weights *w, const float *rope,
+                              int rope_max_pos, wan_stream_t stream);
+
 /* wan_attention -- softmax attention, non-causal, every head
  * ([WALK] self-attention snippet: global window, key lengths).
  *   B, heads, Lq, Lk, head_dim   sizes (head_dim 128 for WAN_BF16; 32, 64

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(PKG, "libwan.so")
 
 WAN_OK, WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED, WAN_ECUDA, WAN_ETIMEOUT = 0, -1, -2, -3, -4, -5
 WAN_F32, WAN_BF16 = 0, 1
+WAN_NOALLOC_WORKSPACE_BYTES = 16 << 20
 (WAN_WS_ACT, WAN_WS_QKV, WAN_WS_O, WAN_WS_QC, WAN_WS_KVC, WAN_WS_OC, WAN_WS_H, WAN_WS_MOD,
  WAN_WS_STATS) = range(9)
 (WAN_K_GEMM_TC, WAN_K_GEMM_SIMT, WAN_K_ATTN_SELF, WAN_K_ATTN_CROSS, WAN_K_ATTN_SIMT, WAN_K_LAYERNORM,
@@ -57,6 +58,8 @@ _SIGS = {
     "wan_block_workspace_offset": (_sz, [ctypes.POINTER(wan_dims), _c_int, _c_int]),
     "wan_block_forward": (_c_int, [ctypes.POINTER(wan_dims), _c_int, _vp, _vp, _vp, _vp,
                                    ctypes.POINTER(wan_block_weights), _vp, _c_int, _vp, _sz, _vp]),
+    "wan_block_forward_noalloc": (_c_int, [ctypes.POINTER(wan_dims), _c_int, _vp, _vp, _vp, _vp,
+                                           ctypes.POINTER(wan_block_weights), _vp, _c_int, _vp]),
     "wan_attention": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
                                _vp, ctypes.c_float, ctypes.POINTER(ctypes.c_int), _vp, _c_int, _vp]),
     "wan_euler_cfg_step": (_c_int, [_vp, _vp, _vp, _c_int, _sz, ctypes.c_float, ctypes.c_float,
@@ -117,6 +120,11 @@ def wan_block_forward(dims, B, x, ctx, ctx_lens, e0, weights, rope, rope_max_pos
     return load().wan_block_forward(ctypes.byref(dims), B, x, ctx, ctx_lens, e0,
                                     ctypes.byref(weights), rope, rope_max_pos, workspace,
                                     ws_bytes, stream)
+
+
+def wan_block_forward_noalloc(dims, B, x, ctx, ctx_lens, e0, weights, rope, rope_max_pos, stream):
+    return load().wan_block_forward_noalloc(ctypes.byref(dims), B, x, ctx, ctx_lens, e0,
+                                            ctypes.byref(weights), rope, rope_max_pos, stream)
 
 
 def wan_attention(B, heads, Lq, Lk, head_dim, dtype, q, k, v, o, k_lens, scale, grid, rope,
