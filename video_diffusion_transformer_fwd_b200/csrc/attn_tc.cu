@@ -32,7 +32,7 @@ constexpr int TK = 128;                // keys per tile
 constexpr int NSLOT = 4;               // K/V ring slots
 constexpr int TILE_BYTES = 128 * D * 2;  // 32 KB: one Q, K or V tile (two 64-column boxes)
 constexpr int BOX_BYTES = TILE_BYTES / 2;
-constexpr int THREADS = 320;
+constexpr int THREADS = 320;                // 8 softmax warps + MMA warp + TMA warp
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_S = idesc_bf16(TQ, TK, 0);
 constexpr uint32_t IDESC_O = idesc_bf16(TQ, D, 1);
@@ -51,6 +51,50 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Two fp32 lanes per instruction (Blackwell packed f32x2 arithmetic).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for x in [-125, 8] on the FMA pipe (Cody-Waite style split, our own
+// near-minimax cubic): r = rint(x) via the 1.5 * 2^23 rounding constant,
+// f = x - r in [-0.5, 0.5], 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 (max relative
+// error 8.4e-5, fitted by iteratively reweighted least squares), and 2^r is
+// added into the exponent field. Inputs below -125 are clamped (2^-125 ~ 0
+// for a bf16 probability).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float2 lo = make_float2(-125.f, -125.f);
+  x = make_float2(fmaxf(x.x, lo.x), fmaxf(x.y, lo.y));
+  const float2 big = make_float2(12582912.f, 12582912.f);       // 1.5 * 2^23
+  const float2 t = fadd2(x, big);
+  const float2 r = fadd2(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = fadd2(x, make_float2(-r.x, -r.y));
+  float2 q = ffma2(make_float2(0.05521299f, 0.05521299f), f, make_float2(0.24271414f, 0.24271414f));
+  q = ffma2(q, f, make_float2(0.69326216f, 0.69326216f));
+  q = ffma2(q, f, make_float2(0.9999196f, 0.9999196f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -111,79 +155,107 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 9) {
-    // ------------------------------------------------ TMA producer
-    if (lane == 0 && nkt > 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      const uint32_t qb = smem_u32(q_full);
-      mbar_arrive_expect_tx(qb, 2 * TILE_BYTES);
-      for (int i = 0; i < 2; ++i)
-        for (int half = 0; half < 2; ++half)
-          tma_load_3d(smem_u32(sQ + i * TILE_BYTES + half * BOX_BYTES), &tmQ, h * D + half * 64,
-                      q0 + i * TQ, b, qb);
-      int slot = 0;
-      uint32_t phase = 0;
-      int fills[NSLOT] = {0, 0, 0, 0};
-      bool ok = true;
-      for (int j = 0; j < nkt && ok; ++j) {
-        for (int kv = 0; kv < 2; ++kv) {
-          if (!mbar_wait(smem_u32(&kv_empty[slot]), phase ^ 1, abort_flag, p.watchdog, 0x201)) { ok = false; break; }
-          const uint32_t fb = smem_u32(&kv_full[slot]);
-          mbar_arrive_expect_tx(fb, TILE_BYTES);
-          const CUtensorMap *tm = kv == 0 ? &tmK : &tmV;
+  if (warp >= 8) {
+    if (warp == 9) {
+      // ------------------------------------------------ TMA producer
+      if (lane == 0 && nkt > 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        const uint32_t qb = smem_u32(q_full);
+        mbar_arrive_expect_tx(qb, 2 * TILE_BYTES);
+        for (int i = 0; i < 2; ++i)
           for (int half = 0; half < 2; ++half)
-            tma_load_3d(smem_u32(sKV + slot * TILE_BYTES + half * BOX_BYTES), tm, h * D + half * 64,
-                        j * TK, b, fb);
-          ++fills[slot];
-          if (++slot == NSLOT) { slot = 0; phase ^= 1; }
+            tma_load_3d(smem_u32(sQ + i * TILE_BYTES + half * BOX_BYTES), &tmQ, h * D + half * 64,
+                        q0 + i * TQ, b, qb);
+        int slot = 0;
+        uint32_t phase = 0;
+        int fills[NSLOT] = {0, 0, 0, 0};
+        bool ok = true;
+        for (int j = 0; j < nkt && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            if (!mbar_wait(smem_u32(&kv_empty[slot]), phase ^ 1, abort_flag, p.watchdog, 0x201)) { ok = false; break; }
+            const uint32_t fb = smem_u32(&kv_full[slot]);
+            mbar_arrive_expect_tx(fb, TILE_BYTES);
+            const CUtensorMap *tm = kv == 0 ? &tmK : &tmV;
+            for (int half = 0; half < 2; ++half)
+              tma_load_3d(smem_u32(sKV + slot * TILE_BYTES + half * BOX_BYTES), tm, h * D + half * 64,
+                          j * TK, b, fb);
+            ++fills[slot];
+            if (++slot == NSLOT) { slot = 0; phase ^= 1; }
+          }
         }
+        int never = 0;
+        mbar_wait(qb, 0, &never, p.watchdog, 0x202);
+        for (int s = 0; s < NSLOT; ++s)
+          if (fills[s] > 0) mbar_wait(smem_u32(&kv_full[s]), (fills[s] - 1) & 1, &never, p.watchdog, 0x203);
       }
-      int never = 0;
-      mbar_wait(qb, 0, &never, p.watchdog, 0x202);
-      for (int s = 0; s < NSLOT; ++s)
-        if (fills[s] > 0) mbar_wait(smem_u32(&kv_full[s]), (fills[s] - 1) & 1, &never, p.watchdog, 0x203);
-    }
-  } else if (warp == 8) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0 && nkt > 0) {
-      bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.watchdog, 0x211);
-      int slot = 0;
-      uint32_t phase = 0;
-      for (int j = 0; j < nkt && ok; ++j) {
-        // S_i = Q_i K_j^T
-        if (!mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x212)) break;
-        const uint32_t kbase = smem_u32(sKV + slot * TILE_BYTES);
-        for (int i = 0; i < 2 && ok; ++i) {
-          if (j > 0 && !mbar_wait(smem_u32(&pv_done[i]), (j - 1) & 1, abort_flag, p.watchdog, 0x213)) { ok = false; break; }
-          tc_fence_after();
+    } else if (warp == 8) {
+      // ------------------------------------------------ MMA issuer
+      if (lane == 0 && nkt > 0) {
+        // Issue order per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1). A
+        // tile's next S reuses the TMEM columns its P occupies; tcgen05.mma ops
+        // of one CTA execute in issue order, so S_i(j+1) is issued right behind
+        // PV_i(j) and each query tile only waits for its own softmax.
+        bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.watchdog, 0x211);
+        int slot = 0;
+        uint32_t phase = 0;
+        auto next = [&]() { if (++slot == NSLOT) { slot = 0; phase ^= 1; } };
+        auto issue_s = [&](int i, uint32_t kbase) {
           const uint32_t qbase = smem_u32(sQ + i * TILE_BYTES);
-#pragma unroll
+  #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
             mma_ss(tmem + i * TK, desc_kmajor_sw128(qbase + off), desc_kmajor_sw128(kbase + off), IDESC_S, kk > 0);
           }
           tc_commit(smem_u32(&s_full[i]));
-        }
-        if (!ok) break;
-        tc_commit(smem_u32(&kv_empty[slot]));
-        if (++slot == NSLOT) { slot = 0; phase ^= 1; }
-        // O_i += P_i V_j
-        if (!mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x214)) break;
-        const uint32_t vbase = smem_u32(sKV + slot * TILE_BYTES);
-        for (int i = 0; i < 2 && ok; ++i) {
-          if (!mbar_wait(smem_u32(&p_ready[i]), j & 1, abort_flag, p.watchdog, 0x215)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
+        };
+        auto issue_pv = [&](int i, uint32_t vbase, int j) {
+  #pragma unroll
           for (int kk = 0; kk < TK / 16; ++kk)
             mma_ts(tmem + 2 * TK + i * D, tmem + i * TK + kk * 8,
                    desc_mnmajor_sw128(vbase + kk * 16 * 128, BOX_BYTES, 1024), IDESC_O, (j > 0 || kk > 0));
           tc_commit(smem_u32(&pv_done[i]));
+        };
+        // prologue: S_0(0), S_1(0)
+        int kslot = slot;
+        if (ok && mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x212)) {
+          tc_fence_after();
+          const uint32_t kbase = smem_u32(sKV + slot * TILE_BYTES);
+          issue_s(0, kbase);
+          issue_s(1, kbase);
+          tc_commit(smem_u32(&kv_empty[kslot]));
+          next();
+        } else {
+          ok = false;
         }
-        if (!ok) break;
-        tc_commit(smem_u32(&kv_empty[slot]));
-        if (++slot == NSLOT) { slot = 0; phase ^= 1; }
+        for (int j = 0; j < nkt && ok; ++j) {
+          if (!mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x214)) break;   // V_j
+          const int vslot = slot;
+          const uint32_t vbase = smem_u32(sKV + slot * TILE_BYTES);
+          next();
+          const bool more = j + 1 < nkt;
+          uint32_t kbase = 0;
+          kslot = slot;
+          if (!mbar_wait(smem_u32(&p_ready[0]), j & 1, abort_flag, p.watchdog, 0x215)) break;
+          tc_fence_after();
+          issue_pv(0, vbase, j);
+          if (more) {
+            if (!mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x216)) break;   // K_{j+1}
+            tc_fence_after();
+            kbase = smem_u32(sKV + slot * TILE_BYTES);
+            next();
+            issue_s(0, kbase);
+          }
+          if (!mbar_wait(smem_u32(&p_ready[1]), j & 1, abort_flag, p.watchdog, 0x217)) break;
+          tc_fence_after();
+          issue_pv(1, vbase, j);
+          tc_commit(smem_u32(&kv_empty[vslot]));
+          if (more) {
+            issue_s(1, kbase);
+            tc_commit(smem_u32(&kv_empty[kslot]));
+          }
+        }
       }
     }
   } else {
@@ -204,56 +276,70 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
       tmem_ld_wait();
       const int kvalid = kl - j * TK;              // keys of this tile that are valid
-      float tmax = -INFINITY;
+      const bool full_tile = kvalid >= TK;         // uniform across the CTA
+      if (!full_tile) {
 #pragma unroll
-      for (int k = 0; k < 128; ++k) {
-        float x = __uint_as_float(s[k]) * p.c;
-        if (k >= kvalid) x = -INFINITY;
-        s[k] = __float_as_uint(x);
-        tmax = fmaxf(tmax, x);
+        for (int k = 0; k < 128; ++k)
+          if (k >= kvalid) s[k] = 0xff800000u;     // -inf
       }
-      // running max with conditional rescaling of l and O; the TMEM accesses
-      // are warp-collective, so a warp rescales when any of its rows must
+      // row max of the raw scores (the scale c is positive), 3-input max tree
+      float mx[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx[a] = fmax3(__uint_as_float(s[a]), __uint_as_float(s[8 + a]), __uint_as_float(s[16 + a]));
+#pragma unroll
+      for (int k = 24; k < 128; k += 16) {
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx[a] = fmax3(mx[a], __uint_as_float(s[k + a]), __uint_as_float(s[k + 8 + a]));
+      }
+      const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * p.c;
+      // running max; l and O are rescaled only when m grows by more than the
+      // threshold (or on the first tile)
       const bool need = (tmax > m + RESCALE_THRESHOLD) || (m == -INFINITY);
       const float mnew = need ? tmax : m;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ex2(m - mnew) : 1.0f;
-        l *= alpha;
-        if (!mbar_wait(smem_u32(&pv_done[i]), (j - 1) & 1, abort_flag, p.watchdog, 0x222)) ok = false;
-        __syncwarp();
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_addr + c * 32, o);
-          tmem_ld_wait();
-          uint32_t a[16], bq[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            a[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            bq[e] = __float_as_uint(__uint_as_float(o[16 + e]) * alpha);
-          }
-          tmem_st16(o_addr + c * 32, a);
-          tmem_st16(o_addr + c * 32 + 16, bq);
-        }
-        tmem_st_wait();
-      }
+      const float alpha = (need && j > 0) ? ex2(m - mnew) : 1.0f;
       m = mnew;
-      // P = exp2(x - m) as bf16 pairs into the first 64 columns of S_i
-      float rs = 0.f;
+      // P = exp2(s c - m) as bf16 pairs into the first 64 columns of S_i. In
+      // full tiles one pair in four is evaluated on the FMA pipe (polynomial
+      // exp2) to take load off the MUFU unit; the rest uses ex2.approx.
+      const float2 c2 = make_float2(p.c, p.c);
+      const float2 nm2 = make_float2(-m, -m);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(__uint_as_float(s[c * 32 + 2 * e]) - m);
-          const float p1 = ex2(__uint_as_float(s[c * 32 + 2 * e + 1]) - m);
-          rs += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
+          const float2 x = ffma2(make_float2(__uint_as_float(s[c * 32 + 2 * e]), __uint_as_float(s[c * 32 + 2 * e + 1])), c2, nm2);
+          float2 pp;
+          if (full_tile && (e & 3) == 3) {
+            pp = exp2_poly2(x);
+          } else {
+            pp = make_float2(ex2(x.x), ex2(x.y));
+          }
+          if (e & 1) acc1 = fadd2(acc1, pp); else acc0 = fadd2(acc0, pp);
+          pk[e] = pack_bf16(pp.x, pp.y);
         }
         tmem_st16(s_addr + c * 16, pk);
       }
-      l += rs;
+      const float2 acc = fadd2(acc0, acc1);
+      l = l * alpha + (acc.x + acc.y);
+      // O rescale after P is out of registers (the PV MMA of this tile is
+      // only issued after p_ready); TMEM accesses are warp-collective, so a
+      // warp rescales when any of its rows must
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        if (!mbar_wait(smem_u32(&pv_done[i]), (j - 1) & 1, abort_flag, p.watchdog, 0x222)) ok = false;
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o[16];
+          tmem_ld16(o_addr + c * 16, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st16(o_addr + c * 16, o);
+        }
+      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();

@@ -1,19 +1,25 @@
 // Tensor-core GEMM for sm_100a: C = A B^T (+ bias) with fused epilogues,
 // bf16 operands, fp32 accumulation in TMEM.
 //
-// Persistent kernel, one CTA per SM, 128 x 256 output tiles, K in steps of 64:
-//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 per stage into
-//               a 4-stage ring (128-byte swizzle), completion on mbarriers;
-//   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=256,
-//               K=16) x 4 per stage into one of two TMEM accumulators
-//               (2 x 256 fp32 columns), commits free the stage / publish
-//               the accumulator;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..+31 = tile rows), bias, GELU or gated
-//               residual, stores to global; the second accumulator lets the
-//               next tile's MMAs run under this epilogue.
-// Tiles are walked in groups of 16 M-tiles so a wave of CTAs shares A and B
-// panels in L2. Every wait is bounded (sm100::mbar_wait).
+// Persistent kernel on CTA pairs (clusters of 2, one CTA per SM): each pair
+// computes 256 x 256 output tiles with tcgen05.mma.cta_group::2 (M = 256 split
+// 128/128 across the two CTAs' TMEM, N = 256, K = 16), K in steps of 64:
+//   warp 0      TMA producer in both CTAs: this CTA's 128 rows of A and its
+//               half (128 rows) of B per stage into a 6-stage ring
+//               (128-byte swizzle); bytes of both CTAs are counted on the
+//               leader CTA's "full" barrier;
+//   warp 1      MMA issuer (leader CTA only): 4 pair MMAs per stage into one
+//               of two TMEM accumulators (2 x 256 fp32 columns per CTA);
+//               commits free the stage in both CTAs and publish the
+//               accumulator to both CTAs' epilogues;
+//   warps 2..5  epilogue in both CTAs: tcgen05.ld of this CTA's 128 rows
+//               (warp w reads TMEM lanes 32*(w%4)..+31), bias, GELU or gated
+//               residual, stores to global (the residual add x += g*y goes
+//               through a swizzled smem tile and a TMA reduce-add into x);
+//               then a release arrive on the leader's "accumulator empty"
+//               barrier.
+// Tiles are walked in groups of 8 M-tiles (2048 rows) so a wave of pairs
+// shares A and B panels in L2. Every wait is bounded (sm100::mbar_wait).
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -22,15 +28,20 @@ namespace wan {
 namespace {
 using namespace sm100;
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;                   // 16 KB
-constexpr int B_BYTES = BN * BK * 2;                   // 32 KB
+constexpr int BM = 128;                  // rows per CTA (256 per pair)
+constexpr int BN = 256;                  // columns per tile (128 B rows per CTA)
+constexpr int BK = 64;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
-constexpr int GROUP_M = 16;
+constexpr int GROUP_M = 8;               // pair tiles (256 rows) per raster group
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0);
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr uint32_t IDESC = idesc_bf16(2 * BM, BN, 0);
+constexpr int STG_BYTES = 32 * 32 * 4;  // one warp's 32 x 32 fp32 staging tile (128-byte swizzle)
+constexpr int EPI_SMEM = 4 * 2 * STG_BYTES;  // 4 epilogue warps, double-buffered
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_SMEM + 256;
 
 struct TcParams {
   int M, N, K, segN;
@@ -60,23 +71,35 @@ template <int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
-               const TcParams p) {
+               const __grid_constant__ CUtensorMap tmX, const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
   uint8_t *sB = smem + STAGES * A_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  uint8_t *sE = smem + STAGES * STAGE_BYTES;      // epilogue staging (residual epilogue)
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sE + EPI_SMEM);
   uint64_t *full = bars, *empty = bars + STAGES, *tfull = bars + 2 * STAGES, *tempty = bars + 2 * STAGES + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  volatile uint32_t *skip = reinterpret_cast<volatile uint32_t *>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
-  // A CTA that starts after another one gave up a wait skips its work, so a
-  // failed launch ends within a few waits instead of one per CTA.
-  if (threadIdx.x == 0) *abort_flag = (p.watchdog && *reinterpret_cast<volatile int *>(p.watchdog)) ? 1 : 0;
-  __syncthreads();
-  if (*abort_flag) return;
+  // The leader decides for both CTAs whether to skip (a wait of an earlier
+  // CTA already gave up), so the pair always takes the same path. The first
+  // cluster barrier guarantees the peer is running before its shared memory
+  // is written.
+  cluster_sync_all();
+  if (leader && threadIdx.x == 0) {
+    const uint32_t v = (p.watchdog && *reinterpret_cast<volatile int *>(p.watchdog)) ? 1u : 0u;
+    *skip = v;
+    st_shared_cluster_u32(mapa_shared(smem_u32((const void *)skip), 1), v);
+  }
+  cluster_sync_all();
+  if (*skip) return;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -85,7 +108,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 4);
+      mbar_init(smem_u32(&tempty[b]), 8);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -95,51 +118,57 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tma_prefetch_desc(&tmB2);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();               // barrier inits of both CTAs visible before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------ TMA producer
+    // ------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int fills[STAGES] = {0, 0, 0, 0};
+      int fills[STAGES] = {0, 0, 0, 0, 0, 0};
       bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      for (int t = pair; t < p.num_tiles && ok; t += npairs) {
         int mb, nb;
         tile_coords(t, p, mb, nb);
         const int n0 = nb * BN;
         const int seg = n0 / p.segN;
         const CUtensorMap *bm = seg == 0 ? &tmB0 : (seg == 1 ? &tmB1 : &tmB2);
-        const int nn0 = n0 - seg * p.segN;
+        const int a_row = mb * 2 * BM + (int)rank * BM;
+        const int b_row = n0 - seg * p.segN + (int)rank * (BN / 2);
         for (int kb = 0; kb < p.num_k; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.watchdog, 0x101)) { ok = false; break; }
-          const uint32_t fb = smem_u32(&full[stage]);
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          tma_load_2d(smem_u32(sA + stage * A_BYTES), &tmA, kb * BK, mb * BM, fb);
-          tma_load_2d(smem_u32(sB + stage * B_BYTES), bm, kb * BK, nn0, fb);
+          const uint32_t fb_local = smem_u32(&full[stage]);
+          if (leader) mbar_arrive_expect_tx(fb_local, 2 * STAGE_BYTES);
+          const uint32_t fb = mapa_shared(fb_local, 0);
+          tma_load_2d_pair(smem_u32(sA + stage * A_BYTES), &tmA, kb * BK, a_row, fb);
+          tma_load_2d_pair(smem_u32(sB + stage * B_BYTES), bm, kb * BK, b_row, fb);
           ++fills[stage];
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
-      // drain: every issued copy has landed before the CTA may exit
-      int never = 0;
-      for (int s = 0; s < STAGES; ++s)
-        if (fills[s] > 0) mbar_wait(smem_u32(&full[s]), (fills[s] - 1) & 1, &never, p.watchdog, 0x102);
+      // drain (leader): every issued copy of the pair has landed before exit.
+      // The peer's copies complete on the leader's barrier, so the leader's
+      // drain also covers them; the final cluster barrier orders the rest.
+      if (leader) {
+        int never = 0;
+        for (int s = 0; s < STAGES; ++s)
+          if (fills[s] > 0) mbar_wait(smem_u32(&full[s]), (fills[s] - 1) & 1, &never, p.watchdog, 0x102);
+      }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++i) {
+      for (int t = pair; t < p.num_tiles && ok; t += npairs, ++i) {
         const int buf = i & 1;
         const uint32_t acc_phase = (i >> 1) & 1;
         if (!mbar_wait(smem_u32(&tempty[buf]), acc_phase ^ 1, abort_flag, p.watchdog, 0x111)) break;
@@ -152,26 +181,35 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint64_t b0 = desc_kmajor_sw128(smem_u32(sB + stage * B_BYTES));
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_ss(d, a0 + 2 * kk, b0 + 2 * kk, IDESC, (kb | kk) != 0);
-          tc_commit(smem_u32(&empty[stage]));
+            mma_ss_pair(d, a0 + 2 * kk, b0 + 2 * kk, IDESC, (kb | kk) != 0);
+          const uint32_t eb = smem_u32(&empty[stage]);
+          tc_commit_pair(eb);
+          tc_commit_pair(mapa_shared(eb, 1));
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
-        if (ok) tc_commit(smem_u32(&tfull[buf]));
+        if (ok) {
+          const uint32_t fb = smem_u32(&tfull[buf]);
+          tc_commit_pair(fb);
+          tc_commit_pair(mapa_shared(fb, 1));
+        }
       }
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int row = q * 32 + lane;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    int stg_count = 0;
     int i = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++i) {
+    for (int t = pair; t < p.num_tiles; t += npairs, ++i) {
       int mb, nb;
       tile_coords(t, p, mb, nb);
       const int buf = i & 1;
       const uint32_t acc_phase = (i >> 1) & 1;
       if (!mbar_wait(smem_u32(&tfull[buf]), acc_phase, abort_flag, p.watchdog, 0x121)) break;
       tc_fence_after();
-      const int m = mb * BM + row;
+      const int m = mb * 2 * BM + (int)rank * BM + row;
       const int n0 = nb * BN;
       const int seg = n0 / p.segN;
       const __nv_bfloat16 *bias = static_cast<const __nv_bfloat16 *>(p.bias[seg]);
@@ -184,10 +222,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (c == BN / 32 - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+          if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
         }
         const int n = n0 + c * 32;
-        if (m >= p.M || n >= p.N) continue;
+        if (EPI == EPI_RESID) {
+          if (mb * 2 * BM + (int)rank * BM + q * 32 >= p.M || n >= p.N) continue;   // warp-uniform
+        } else if (m >= p.M || n >= p.N) {
+          continue;
+        }
         float v[32];
         const uint4 *bp = reinterpret_cast<const uint4 *>(bias + nn0 + c * 32);
 #pragma unroll
@@ -201,18 +243,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
         }
         if (EPI == EPI_RESID) {
-          float *xr = p.X + (size_t)m * p.ldx + n;
-          const float *gr = p.gate ? p.gate + (size_t)(m / p.rows_per_gate) * p.gate_stride + n : nullptr;
+          // x[m, n..n+31] += g * v through a swizzled shared-memory tile and a
+          // TMA reduce-add (the read-modify-write of x happens in L2; rows
+          // beyond M are clipped by the tensor map)
+          const int m0w = mb * 2 * BM + (int)rank * BM + q * 32;       // warp-uniform
+          const float *gr = (p.gate && m < p.M)
+                                ? p.gate + (size_t)(m / p.rows_per_gate) * p.gate_stride + n : nullptr;
+          uint8_t *buf = sE + ((warp - 2) * 2 + (stg_count & 1)) * STG_BYTES;
+          if (lane == 0) bulk_wait_group_read<1>();      // this buffer's previous reduce has read it
+          __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            float4 xv = *reinterpret_cast<const float4 *>(xr + j);
-            const float4 gv = gr ? *reinterpret_cast<const float4 *>(gr + j) : make_float4(1.f, 1.f, 1.f, 1.f);
-            xv.x = fmaf(gv.x, v[j + 0], xv.x);
-            xv.y = fmaf(gv.y, v[j + 1], xv.y);
-            xv.z = fmaf(gv.z, v[j + 2], xv.z);
-            xv.w = fmaf(gv.w, v[j + 3], xv.w);
-            *reinterpret_cast<float4 *>(xr + j) = xv;
+          for (int j16 = 0; j16 < 8; ++j16) {
+            float4 gv = make_float4(1.f, 1.f, 1.f, 1.f);
+            if (p.gate) gv = gr ? *reinterpret_cast<const float4 *>(gr + 4 * j16) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 o = make_float4(gv.x * v[4 * j16 + 0], gv.y * v[4 * j16 + 1],
+                                         gv.z * v[4 * j16 + 2], gv.w * v[4 * j16 + 3]);
+            *reinterpret_cast<float4 *>(buf + lane * 128 + ((j16 ^ (lane & 7)) << 4)) = o;
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_2d(&tmX, smem_u32(buf), n, m0w);
+            bulk_commit_group();
+          }
+          ++stg_count;
         } else {
           __nv_bfloat16 *cr = static_cast<__nv_bfloat16 *>(p.C) + (size_t)m * p.ldc + n;
 #pragma unroll
@@ -236,23 +290,46 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
   }
 
+  if (EPI == EPI_RESID && warp >= 2 && lane == 0) bulk_wait_group_all();   // reduces done with smem
+
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();               // the peer's smem and TMEM stay live until the leader is done
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
 template <int EPI>
-int launch(const CUtensorMap &ta, const CUtensorMap *tb, const TcParams &p, cudaStream_t s) {
-  static bool attr_set = false;     // per process; the attribute is per function
-  if (!attr_set) {
+int launch(const CUtensorMap &ta, const CUtensorMap *tb, const CUtensorMap &tx, const TcParams &p,
+           cudaStream_t s) {
+  static int max_pairs = 0;         // per process; the attribute is per function
+  if (!max_pairs) {
     WAN_TRY_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
                  "gemm_tc smem attribute");
-    attr_set = true;
+    cudaLaunchConfig_t qc = {};
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = 2; qa[0].val.clusterDim.y = 1; qa[0].val.clusterDim.z = 1;
+    qc.gridDim = dim3(2 * 74, 1, 1);
+    qc.blockDim = dim3(THREADS, 1, 1);
+    qc.dynamicSmemBytes = SMEM_BYTES;
+    qc.attrs = qa;
+    qc.numAttrs = 1;
+    int clusters = 0;
+    WAN_TRY_CUDA(cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<EPI>, &qc), "gemm_tc occupancy");
+    max_pairs = clusters > 0 ? clusters : sm_count() / 2;
   }
-  const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
-  gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ta, tb[0], tb[1], tb[2], p);
-  WAN_CHECK_LAUNCH("gemm_tc");
+  const int pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2; attr[0].val.clusterDim.y = 1; attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  WAN_TRY_CUDA(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI>, ta, tb[0], tb[1], tb[2], tx, p), "gemm_tc launch");
   return WAN_OK;
 }
 }  // namespace
@@ -263,7 +340,7 @@ bool gemm_tc_supported(const GemmArgs &g) {
   if (g.nseg > 1 && g.segN % BN) return false;
   if (g.lda % 8) return false;
   if (g.epi != EPI_RESID && g.ldc % 8) return false;
-  if (g.epi == EPI_RESID && (g.ldx % 4 || (g.gate && g.gate_stride % 4))) return false;
+  if (g.epi == EPI_RESID && (g.ldx % 4 || !aligned16(g.X) || (g.gate && g.gate_stride % 4))) return false;
   for (int i = 0; i < g.nseg; ++i)
     if (!aligned16(g.Bseg[i]) || (g.bias[i] && !aligned16(g.bias[i]))) return false;
   return aligned16(g.A);
@@ -276,11 +353,11 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   if (rc) return rc;
   for (int i = 0; i < 3; ++i) {
     const int si = i < g.nseg ? i : 0;
-    if ((rc = encode_tmap_2d_bf16(&tb[i], g.Bseg[si], g.K, g.segN, (uint64_t)g.K * 2, BK, BN))) return rc;
+    if ((rc = encode_tmap_2d_bf16(&tb[i], g.Bseg[si], g.K, g.segN, (uint64_t)g.K * 2, BK, BN / 2))) return rc;
   }
   TcParams p = {};
   p.M = g.M; p.N = g.N; p.K = g.K; p.segN = g.segN;
-  p.num_m = (g.M + BM - 1) / BM;
+  p.num_m = (g.M + 2 * BM - 1) / (2 * BM);
   p.num_n = (g.N + BN - 1) / BN;
   p.num_tiles = p.num_m * p.num_n;
   p.num_k = g.K / BK;
@@ -288,10 +365,12 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   p.C = g.C; p.ldc = g.ldc; p.X = g.X; p.ldx = g.ldx;
   p.gate = g.gate; p.gate_stride = g.gate_stride; p.rows_per_gate = g.rows_per_gate > 0 ? g.rows_per_gate : 1;
   p.watchdog = watchdog_ptr();
+  CUtensorMap tx = ta;
+  if (g.epi == EPI_RESID && (rc = encode_tmap_2d_f32(&tx, g.X, g.N, g.M, (uint64_t)g.ldx * 4, 32, 32))) return rc;
   switch (g.epi) {
-    case EPI_STORE: return launch<EPI_STORE>(ta, tb, p, s);
-    case EPI_GELU: return launch<EPI_GELU>(ta, tb, p, s);
-    default: return launch<EPI_RESID>(ta, tb, p, s);
+    case EPI_STORE: return launch<EPI_STORE>(ta, tb, tx, p, s);
+    case EPI_GELU: return launch<EPI_GELU>(ta, tb, tx, p, s);
+    default: return launch<EPI_RESID>(ta, tb, tx, p, s);
   }
 }
 
