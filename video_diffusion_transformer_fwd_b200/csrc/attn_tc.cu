@@ -77,26 +77,6 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
-// 2^x for x in [-125, 8] on the FMA pipe (Cody-Waite style split, our own
-// near-minimax cubic): r = rint(x) via the 1.5 * 2^23 rounding constant,
-// f = x - r in [-0.5, 0.5], 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 (max relative
-// error 8.4e-5, fitted by iteratively reweighted least squares), and 2^r is
-// added into the exponent field. Inputs below -125 are clamped (2^-125 ~ 0
-// for a bf16 probability).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  const float2 lo = make_float2(-125.f, -125.f);
-  x = make_float2(fmaxf(x.x, lo.x), fmaxf(x.y, lo.y));
-  const float2 big = make_float2(12582912.f, 12582912.f);       // 1.5 * 2^23
-  const float2 t = fadd2(x, big);
-  const float2 r = fadd2(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = fadd2(x, make_float2(-r.x, -r.y));
-  float2 q = ffma2(make_float2(0.05521299f, 0.05521299f), f, make_float2(0.24271414f, 0.24271414f));
-  q = ffma2(q, f, make_float2(0.69326216f, 0.69326216f));
-  q = ffma2(q, f, make_float2(0.9999196f, 0.9999196f));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
@@ -298,9 +278,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float mnew = need ? tmax : m;
       const float alpha = (need && j > 0) ? ex2(m - mnew) : 1.0f;
       m = mnew;
-      // P = exp2(s c - m) as bf16 pairs into the first 64 columns of S_i. In
-      // full tiles one pair in four is evaluated on the FMA pipe (polynomial
-      // exp2) to take load off the MUFU unit; the rest uses ex2.approx.
+      // P = exp2(s c - m) as bf16 pairs into the first 64 columns of S_i
+      // (ex2.approx on the MUFU unit; measured, it is not the limiter here).
       const float2 c2 = make_float2(p.c, p.c);
       const float2 nm2 = make_float2(-m, -m);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
@@ -310,12 +289,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float2 x = ffma2(make_float2(__uint_as_float(s[c * 32 + 2 * e]), __uint_as_float(s[c * 32 + 2 * e + 1])), c2, nm2);
-          float2 pp;
-          if (full_tile && (e & 3) == 3) {
-            pp = exp2_poly2(x);
-          } else {
-            pp = make_float2(ex2(x.x), ex2(x.y));
-          }
+          const float2 pp = make_float2(ex2(x.x), ex2(x.y));
           if (e & 1) acc1 = fadd2(acc1, pp); else acc0 = fadd2(acc0, pp);
           pk[e] = pack_bf16(pp.x, pp.y);
         }
