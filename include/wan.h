@@ -210,6 +210,15 @@ int wan_euler_cfg_step(float *x, const void *v_cond, const void *v_uncond,
  * outputs are then invalid), or WAN_ECUDA if the stream holds a CUDA error. */
 int wan_device_status(wan_stream_t stream);
 
+/* wan_selftest_watchdog -- enqueue a one-CTA kernel whose bounded wait on an
+ * mbarrier can never complete, so the wait gives up after its limit (about
+ * 2 s), records its code in the watchdog word and returns without trapping.
+ * A following wan_device_status(stream) reports WAN_ETIMEOUT (and clears the
+ * word); the CUDA context stays usable. Test support for the failure path of
+ * every tcgen05 kernel's waits; the pages have no counterpart. While the word
+ * is set, tensor-core kernels launched afterwards skip their work. */
+int wan_selftest_watchdog(wan_stream_t stream);
+
 /* Launch instrumentation. While enabled, every kernel the library launches is
  * bracketed by two CUDA events recorded on its stream (a few microseconds of
  * host overhead per launch). wan_profile_enable(on) also clears the record;

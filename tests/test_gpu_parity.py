@@ -238,3 +238,41 @@ def test_block_1p3b_long_f32_pass():
     ref = run.oracle_rows(rows)
     got = np64(run.x[:, torch.as_tensor(rows, device="cuda")])
     assert np.abs(got - ref).max() <= F32_MAX_ABS
+
+
+# ------------------------------------------------------------------ failure path, full-size step
+
+def test_watchdog_wait_expires_and_context_survives():
+    """A bounded wait that can never complete gives up, the host reads
+    WAN_ETIMEOUT, and the next library call still works."""
+    s = torch.cuda.current_stream().cuda_stream
+    wan.check(wan.wan_selftest_watchdog(s))
+    assert wan.wan_device_status(s) == wan.WAN_ETIMEOUT
+    assert wan.wan_device_status(s) == wan.WAN_OK            # the status was cleared
+    got, ref = _attn_case(1, 130, 200, 2, 128, "bf16")       # tensor-core path runs again
+    assert rel_l2(got, ref) <= BF16_REL_L2
+
+
+def test_a14b_step_full_size_identity():
+    """The full-size A14B step (40 blocks, CFG pair, L = 32760) in the bench's
+    launch sequence, with every gate and the cross-attention output projection
+    zeroed: each block is then exactly the identity, so v_c = v_u = x and the
+    step is x + (sigma' - sigma) x."""
+    from video_diffusion_transformer_fwd_b200.step import DenoiseStep
+    cfg = configs.get("a14b-step")
+    st = DenoiseStep(cfg, seed=7)
+    for w in st.weights:
+        w["modulation"][2].zero_()
+        w["modulation"][5].zero_()
+        w["cwo"].zero_()
+        w["cbo"].zero_()
+    st.e0[:, 2].zero_()
+    st.e0[:, 5].zero_()
+    x0 = st.x.clone()
+    st.step()
+    torch.cuda.synchronize()
+    assert wan.device_status() == wan.WAN_OK
+    assert torch.equal(st.xb[0], x0) and torch.equal(st.xb[1], x0)
+    dt = float(np.float32(cfg.sigma_next) - np.float32(cfg.sigma))
+    ref = O.euler_cfg_step(np64(x0), np64(x0), np64(x0), cfg.guide_scale, 0.0, dt)
+    assert np.abs(np64(st.x) - ref).max() <= 1e-5

@@ -66,6 +66,7 @@ _SIGS = {
                                     ctypes.c_float, _vp]),
     "wan_device_status": (_c_int, [_vp]),
     "wan_profile_enable": (_c_int, [_c_int]),
+    "wan_selftest_watchdog": (_c_int, [_vp]),
     "wan_profile_read": (_c_int, [_c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]),
 }
 
@@ -141,6 +142,10 @@ def wan_euler_cfg_step(x, v_cond, v_uncond, v_dtype, n, guide_scale, sigma, sigm
 
 def wan_device_status(stream):
     return load().wan_device_status(stream)
+
+
+def wan_selftest_watchdog(stream):
+    return load().wan_selftest_watchdog(stream)
 
 
 def wan_profile_enable(on):
