@@ -188,6 +188,24 @@ def blas_threads():
         return None
 
 
+# ----------------------------------------------------------------- multi-rank timing
+def max_over_ranks(ms: float, world: int, device="cpu") -> float:
+    """Max of a per-rank device time over all ranks (the job's time)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def per_block_ms(job_ms: float, steps: int, blocks: int, world: int) -> float:
+    """Whole-job ms per block forward of one sequence: every rank runs `steps`
+    steps of `blocks` blocks on the CFG pair (2 sequences)."""
+    return job_ms / (steps * blocks * 2 * world)
+
+
 # ----------------------------------------------------------------- reference arm
 def run_reference(args, rank, world):
     if rank != 0:
@@ -273,10 +291,7 @@ def run_ours(args, rank, world, local_rank):
     if wan.device_status() != wan.WAN_OK:
         raise RuntimeError("timed region: " + wan.last_error())
 
-    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms_total, world, dev)
 
     # end to end: host (pinned) inputs in, result out, every step
     e2e = None
@@ -304,17 +319,13 @@ def run_ours(args, rank, world, local_rank):
         e_end.record(stream)
         torch.cuda.synchronize()
         barrier()
-        te = torch.tensor([e_start.elapsed_time(e_end)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        units = args.steps * cfg.blocks * 2 * world
-        e2e = {"value": float(te.item()) / units, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, dev)
+        e2e = {"value": per_block_ms(e_ms, args.steps, cfg.blocks, world), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
 
     if rank != 0:
         return
-    units = args.steps * cfg.blocks * 2 * world
-    value = ms_max / units
+    value = per_block_ms(ms_max, args.steps, cfg.blocks, world)
     peaks, peak_src = read_peaks()
     blocks_run = args.steps * cfg.blocks
     import dataclasses

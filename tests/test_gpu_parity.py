@@ -158,6 +158,15 @@ def test_block_is_deterministic():
     assert torch.equal(a.x, b.x)
 
 
+def test_block_bf16_is_deterministic():
+    """The tensor-core path (including the TMA reduce-add residual) gives
+    bit-identical results run to run."""
+    cfg = BlockConfig("bf16-det", 3, 5, 7, 512, 4, 1024, 24, "bf16")
+    a = GpuBlockRun(cfg, B=2, seed=13).run()
+    b = GpuBlockRun(cfg, B=2, seed=13).run()
+    assert torch.equal(a.x, b.x)
+
+
 def test_tiny_stack_of_40_blocks_and_step():
     """The denoising-step launch sequence (40 blocks on the CFG pair, then
     CFG-Euler) on the tiny config, against the full fp64 chain."""
