@@ -41,7 +41,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 TRAFFIC = {
     # profiles/attn_tc_B1_L16384.md: 653.4 MB per launch at B=1, L=16384, scaled by the
     # query/key rows (x4) to the step's launch at B=2, L=32760
-    "attn_self": {"bytes_per_launch": 4 * 653.4e6, "source_sha": "3778302a0827fe60"},
+    "attn_self": {"bytes_per_launch": 4 * 653.4e6, "source_sha": "stale: recapture"},
 }
 
 
@@ -66,10 +66,16 @@ def read_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash(name):
-    p = os.path.join(ROOT, "video_diffusion_transformer_fwd_b200", "csrc", name)
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_hash(*names):
+    """Hash of the sources a kernel is compiled from (its .cu and the shared headers)."""
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "video_diffusion_transformer_fwd_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+ATTN_SOURCES = ("attn_tc.cu", "sm100.cuh", "common.cuh")
 
 
 # ----------------------------------------------------------------- clocks
@@ -343,7 +349,7 @@ def run_ours(args, rank, world, local_rank):
         avg_ms = attn_ms / attn_n
         tr = TRAFFIC.get("attn_self")
         traffic = None
-        if tr and tr.get("source_sha") == source_hash("attn_tc.cu"):
+        if tr and tr.get("source_sha") == source_hash(*ATTN_SOURCES):
             traffic = tr["bytes_per_launch"]
         roofline = {"kernel": "attn_tc (self-attention, B=2, L=32760, 40 heads, d=128)",
                     "bound": "tensor", "achieved": attn_flops_launch / (avg_ms * 1e-3) / 1e12,

@@ -57,20 +57,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase of parity `parity` to complete. Gives up after
 // WAIT_LIMIT_NS or when another thread of the CTA has raised `*abort`; on
 // giving up it records `code` in the library's watchdog word and raises
-// `*abort`, and returns false. Never traps.
-static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                       int *watchdog, int code) {
+// `*abort`, and returns false. Never traps. Inlined: the common case (phase
+// already complete, or completing while try_wait suspends the thread) costs
+// one instruction; the timer and the abort flag are checked every 16 tries.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
+                                          int *watchdog, int code) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  while (true) {
+  unsigned long long t0 = 0;
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer() - t0 > WAIT_LIMIT_NS) {
-      if (watchdog) atomicExch(watchdog, code);
-      *abort = 1;
-      return false;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15) == 0) {
+      if (*abort) return false;
+      const unsigned long long t = globaltimer();
+      if (t0 == 0) {
+        t0 = t;
+      } else if (t - t0 > WAIT_LIMIT_NS) {
+        if (watchdog) atomicExch(watchdog, code);
+        *abort = 1;
+        return false;
+      }
     }
   }
 }
