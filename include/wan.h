@@ -105,14 +105,16 @@ size_t wan_block_workspace_bytes(const wan_dims *dims, int B);
 
 /* Workspace buffers (for inspection after a call; all row-major):          */
 #define WAN_WS_ACT   0  /* (dt) [B*L, dim]   last normalised branch input (FFN's)  */
-#define WAN_WS_QKV   1  /* (dt) [B*L, 3*dim] self q | k | v, q/k normalised+rotated */
+#define WAN_WS_QKV   1  /* (dt) [B*L, 3*dim] self q | k | v: k normalised and rotated; q rotated
+                           (on the bf16 path q's RMS factor is applied inside the attention) */
 #define WAN_WS_O     2  /* (dt) [B*L, dim]   self-attention output (before W_o)     */
 #define WAN_WS_QC    3  /* (dt) [B*L, dim]   cross-attention q (normalised)         */
 #define WAN_WS_KVC   4  /* (dt) [B*T, 2*dim] cross k | v (k normalised)             */
 #define WAN_WS_OC    5  /* (dt) [B*L, dim]   cross-attention output (before W_o)    */
 #define WAN_WS_H     6  /* (dt) [B*L, ffn]   FFN hidden after GELU                  */
 #define WAN_WS_MOD   7  /* f32  [B, 6, dim]  modulation + e0                        */
-#define WAN_WS_STATS 8  /* f32  [B*L, 4]     row statistics scratch                 */
+#define WAN_WS_STATS 8  /* f32  [max(B*L, B*T), 4, dim/256] per-row partial sums of squares of
+                           q, k, cross q, cross k (bf16 path) */
 #define WAN_WS_COUNT 9
 /* Byte offset of buffer `which` inside the workspace, or (size_t)-1. */
 size_t wan_block_workspace_offset(const wan_dims *dims, int B, int which);

@@ -100,7 +100,7 @@ static WsLayout layout_of(const wan_dims *d, int B) {
       BL * D * es,            // OC
       BL * Fh * es,           // H
       (size_t)B * 6 * D * 4,  // MOD
-      BL * 4 * 4,             // STATS
+      (BL > (size_t)B * T ? BL : (size_t)B * T) * 4 * (D >= 256 ? D / 256 : 1) * 4,   // STATS: per-row partial sums of squares
   };
   size_t o = 0;
   for (int i = 0; i < WAN_WS_COUNT; ++i) {
@@ -184,24 +184,40 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
   if ((rc = WAN_PROF(WAN_K_MISC, s, launch_mod_combine(w->modulation, e0, mod, B, D, s)))) return rc;
 
   // ---- self-attention branch: x += m2 * Wo . Attn(RoPE(RMSNorm(q,k)), v)
+  // bf16 tensor-core path: the QKV GEMM epilogue accumulates each row's sum of
+  // squares of q and k, writes gamma * RoPE(y); the attention applies q's RMS
+  // factor in its logit scale and a row pass applies k's. Otherwise: plain
+  // GEMM, then an RMSNorm + RoPE pass over q and k.
+  float *stats = reinterpret_cast<float *>(ws + lay.off[WAN_WS_STATS]);
+  GemmArgs gqkv = {};
+  gqkv.M = BL; gqkv.N = 3 * D; gqkv.K = D; gqkv.A = act; gqkv.lda = D;
+  gqkv.Bseg[0] = w->wq; gqkv.Bseg[1] = w->wk; gqkv.Bseg[2] = w->wv;
+  gqkv.bias[0] = w->bq; gqkv.bias[1] = w->bk; gqkv.bias[2] = w->bv;
+  gqkv.segN = D; gqkv.nseg = 3; gqkv.C = qkv; gqkv.ldc = 3 * D;
+  gqkv.epi = EPI_QKNORM;
+  gqkv.gamma[0] = w->gq; gqkv.gamma[1] = w->gk; gqkv.gamma[2] = nullptr;
+  const int parts = D >= 256 ? D / 256 : 1;          // partial sums per row (one per 256-column tile)
+  const int sstride = 4 * parts;                      // q | k | cross q | cross k partials of a row
+  gqkv.ss = stats; gqkv.ss_stride = sstride; gqkv.ss_col[0] = 0; gqkv.ss_col[1] = 1; gqkv.ss_col[2] = -1;
+  gqkv.rope = rope; gqkv.rope_mask = 3; gqkv.F = d.F; gqkv.H = d.H; gqkv.W = d.W; gqkv.head_dim = hd;
+  AttnArgs aself = {};
+  aself.B = B; aself.heads = d.heads; aself.Lq = L; aself.Lk = L; aself.d = hd;
+  aself.q = qkv; aself.ldq = 3 * D; aself.k = qkv + D * es; aself.ldk = 3 * D; aself.v = qkv + 2 * D * es; aself.ldv = 3 * D;
+  aself.o = o; aself.ldo = D; aself.k_lens = nullptr; aself.scale = 1.0f / sqrtf((float)hd);
+  const bool fused = dt == WAN_BF16 && gemm_tc_supported(gqkv) && attention_tc_supported(aself);
+
   if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, L, mod, 0, 1, nullptr, nullptr, d.eps, s)))) return rc;
-  {
-    GemmArgs g = {};
-    g.M = BL; g.N = 3 * D; g.K = D; g.A = act; g.lda = D;
-    g.Bseg[0] = w->wq; g.Bseg[1] = w->wk; g.Bseg[2] = w->wv;
-    g.bias[0] = w->bq; g.bias[1] = w->bk; g.bias[2] = w->bv;
-    g.segN = D; g.nseg = 3; g.epi = EPI_STORE; g.C = qkv; g.ldc = 3 * D;
-    if ((rc = run_gemm(g, dt, s))) return rc;
+  if (fused) {
+    if ((rc = run_gemm(gqkv, dt, s))) return rc;
+    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_scale_rows(qkv + D * es, BL, 3 * D, D, stats + parts, sstride, parts, d.eps, s)))) return rc;
+    aself.q_ss = stats; aself.q_ss_stride = sstride; aself.q_ss_parts = parts; aself.q_ss_n = (float)D; aself.q_ss_eps = d.eps;
+  } else {
+    gqkv.epi = EPI_STORE;
+    if ((rc = run_gemm(gqkv, dt, s))) return rc;
+    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qkv, dt, BL, 3 * D, D, hd, w->gq, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s)))) return rc;
+    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qkv + D * es, dt, BL, 3 * D, D, hd, w->gk, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s)))) return rc;
   }
-  if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qkv, dt, BL, 3 * D, D, hd, w->gq, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s)))) return rc;
-  if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qkv + D * es, dt, BL, 3 * D, D, hd, w->gk, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s)))) return rc;
-  {
-    AttnArgs a = {};
-    a.B = B; a.heads = d.heads; a.Lq = L; a.Lk = L; a.d = hd;
-    a.q = qkv; a.ldq = 3 * D; a.k = qkv + D * es; a.ldk = 3 * D; a.v = qkv + 2 * D * es; a.ldv = 3 * D;
-    a.o = o; a.ldo = D; a.k_lens = nullptr; a.scale = 1.0f / sqrtf((float)hd);
-    if ((rc = run_attention(a, dt, s, WAN_K_ATTN_SELF))) return rc;
-  }
+  if ((rc = run_attention(aself, dt, s, WAN_K_ATTN_SELF))) return rc;
   {
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = D; g.A = o; g.lda = D;
@@ -216,23 +232,36 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = D; g.A = act; g.lda = D;
     g.Bseg[0] = w->cwq; g.bias[0] = w->cbq; g.segN = D; g.nseg = 1;
-    g.epi = EPI_STORE; g.C = qc; g.ldc = D;
+    g.C = qc; g.ldc = D;
+    g.epi = fused ? EPI_QKNORM : EPI_STORE;
+    g.gamma[0] = w->cgq; g.ss = stats; g.ss_stride = sstride; g.ss_col[0] = 2; g.ss_col[1] = g.ss_col[2] = -1;
     if ((rc = run_gemm(g, dt, s))) return rc;
   }
-  if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qc, dt, BL, D, D, hd, w->cgq, d.eps, nullptr, 0, 1, 1, 1, s)))) return rc;
+  if (!fused && (rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qc, dt, BL, D, D, hd, w->cgq, d.eps, nullptr, 0, 1, 1, 1, s)))) return rc;
   if (T > 0) {
     GemmArgs g = {};
     g.M = B * T; g.N = 2 * D; g.K = D; g.A = ctx; g.lda = D;
     g.Bseg[0] = w->cwk; g.Bseg[1] = w->cwv; g.bias[0] = w->cbk; g.bias[1] = w->cbv;
-    g.segN = D; g.nseg = 2; g.epi = EPI_STORE; g.C = kvc; g.ldc = 2 * D;
+    g.segN = D; g.nseg = 2; g.C = kvc; g.ldc = 2 * D;
+    g.epi = fused ? EPI_QKNORM : EPI_STORE;
+    g.gamma[0] = w->cgk; g.gamma[1] = nullptr; g.ss = stats; g.ss_stride = sstride;
+    g.ss_col[0] = 3; g.ss_col[1] = -1; g.ss_col[2] = -1;
     if ((rc = run_gemm(g, dt, s))) return rc;
-    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(kvc, dt, B * T, 2 * D, D, hd, w->cgk, d.eps, nullptr, 0, 1, 1, 1, s)))) return rc;
+    if (fused) {
+      if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_scale_rows(kvc, B * T, 2 * D, D, stats + 3 * parts, sstride, parts, d.eps, s)))) return rc;
+    } else if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(kvc, dt, B * T, 2 * D, D, hd, w->cgk, d.eps, nullptr, 0, 1, 1, 1, s)))) {
+      return rc;
+    }
   }
   {
     AttnArgs a = {};
     a.B = B; a.heads = d.heads; a.Lq = L; a.Lk = T; a.d = hd;
     a.q = qc; a.ldq = D; a.k = kvc; a.ldk = 2 * D; a.v = kvc + D * es; a.ldv = 2 * D;
     a.o = oc; a.ldo = D; a.k_lens = ctx_lens; a.scale = 1.0f / sqrtf((float)hd);
+    if (fused) {
+      a.q_ss = stats + 2 * parts; a.q_ss_stride = sstride; a.q_ss_parts = parts;
+      a.q_ss_n = (float)D; a.q_ss_eps = d.eps;
+    }
     if ((rc = run_attention(a, dt, s, WAN_K_ATTN_CROSS))) return rc;
   }
   {

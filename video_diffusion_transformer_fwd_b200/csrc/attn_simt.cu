@@ -34,9 +34,17 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(const AttnArgs a) {
 
   float4 q[NC], o[NC];
   const T *qrow = Q + (size_t)(b * a.Lq + (active ? r : 0)) * a.ldq + h * D;
+  // optional per-row RMS factor of q (q left un-normalised by its producer)
+  float qs = 1.0f;
+  if (a.q_ss && active) {
+    float sum = 0.f;
+    for (int t = 0; t < a.q_ss_parts; ++t) sum += a.q_ss[(size_t)(b * a.Lq + r) * a.q_ss_stride + t];
+    qs = 1.0f / sqrtf(sum / a.q_ss_n + a.q_ss_eps);
+  }
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
     q[c] = active ? load4(qrow + 16 * c + 4 * part) : make_float4(0.f, 0.f, 0.f, 0.f);
+    q[c].x *= qs; q[c].y *= qs; q[c].z *= qs; q[c].w *= qs;
     o[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   float m = -INFINITY, l = 0.f;

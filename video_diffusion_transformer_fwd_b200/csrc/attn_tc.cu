@@ -44,6 +44,7 @@ struct FaParams {
   const int *k_lens;
   float c;                    // scale * log2(e)
   __nv_bfloat16 *o; int ldo;
+  const float *q_ss; int q_ss_stride; int q_ss_parts; float q_ss_inv_n; float q_ss_eps;   // optional per-row RMS factor of q
   int *watchdog;
 };
 
@@ -247,6 +248,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const uint32_t s_addr = tmem + lane_off + i * TK;
     const uint32_t o_addr = tmem + lane_off + 2 * TK + i * D;
     float m = -INFINITY, l = 0.f;
+    // logit scale of this row: scale * log2(e), times q's RMS factor when the
+    // QKV epilogue left q un-normalised (q_ss holds the row's sum of squares)
+    float crow = p.c;
+    if (p.q_ss && row < p.Lq) {
+      const float *qs = p.q_ss + (size_t)(b * p.Lq + row) * p.q_ss_stride;
+      float sum = 0.f;
+      for (int t = 0; t < p.q_ss_parts; ++t) sum += qs[t];
+      crow *= rsqrtf(sum * p.q_ss_inv_n + p.q_ss_eps);
+    }
     bool ok = true;
     for (int j = 0; j < nkt; ++j) {
       if (!mbar_wait(smem_u32(&s_full[i]), j & 1, abort_flag, p.watchdog, 0x221)) { ok = false; break; }
@@ -271,7 +281,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int a = 0; a < 8; ++a) mx[a] = fmax3(mx[a], __uint_as_float(s[k + a]), __uint_as_float(s[k + 8 + a]));
       }
-      const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * p.c;
+      const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * crow;
       // running max; l and O are rescaled only when m grows by more than the
       // threshold (or on the first tile)
       const bool need = (tmax > m + RESCALE_THRESHOLD) || (m == -INFINITY);
@@ -280,7 +290,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       m = mnew;
       // P = exp2(s c - m) as bf16 pairs into the first 64 columns of S_i
       // (ex2.approx on the MUFU unit; measured, it is not the limiter here).
-      const float2 c2 = make_float2(p.c, p.c);
+      const float2 c2 = make_float2(crow, crow);
       const float2 nm2 = make_float2(-m, -m);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -385,6 +395,8 @@ int attention_tc(const AttnArgs &a, cudaStream_t s) {
   FaParams p = {};
   p.B = a.B; p.heads = a.heads; p.Lq = a.Lq; p.Lk = a.Lk; p.k_lens = a.k_lens;
   p.c = a.scale * 1.4426950408889634f;
+  p.q_ss = a.q_ss; p.q_ss_stride = a.q_ss_stride; p.q_ss_parts = a.q_ss_parts;
+  p.q_ss_inv_n = a.q_ss_n > 0.f ? 1.0f / a.q_ss_n : 0.f; p.q_ss_eps = a.q_ss_eps;
   p.o = static_cast<__nv_bfloat16 *>(a.o); p.ldo = a.ldo;
   p.watchdog = watchdog_ptr();
   dim3 grid((a.Lq + 2 * TQ - 1) / (2 * TQ), a.heads, a.B);

@@ -93,7 +93,7 @@ inline size_t dtype_size(int dt) { return dt == WAN_BF16 ? 2 : 4; }
 
 // ---------------------------------------------------------------- internal kernels API
 
-enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2 };
+enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_QKNORM = 3 };
 
 // C = A B^T (+ bias) with a fused epilogue. A [M,K] row-major (lda),
 // B given as up to 3 row-major segments [segN, K] (ldb = K) stacked along N,
@@ -102,6 +102,13 @@ enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2 };
 //   EPI_GELU:  C[m,n] = gelu_tanh(acc + bias)
 //   EPI_RESID: X[m,n] += g * (acc + bias), g = gate[(m / rows_per_gate) *
 //              gate_stride + n] or 1 when gate == NULL  (X float32, ldx)
+//   EPI_QKNORM (tensor-core path): per segment s, y = acc + bias; when
+//              ss_col[s] >= 0, the sum of y^2 over each 256-column tile t of the
+//              segment is written to ss[m * ss_stride + ss_col[s] * (segN / 256) + t]
+//              (the consumer adds the segN / 256 partials of a row),
+//              and C = gamma[s] * y, rotated by the 3D RoPE of token m % L when
+//              bit s of rope_mask is set; otherwise C = y. The row's RMS factor
+//              is applied later (attention logit scale for q, a row pass for k).
 struct GemmArgs {
   int M, N, K;
   const void *A; int lda;
@@ -110,6 +117,8 @@ struct GemmArgs {
   void *C; int ldc;
   float *X; int ldx;
   const float *gate; int gate_stride; int rows_per_gate;
+  const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
+  const float *rope; int rope_mask; int F, H, W; int head_dim;
 };
 
 int gemm_simt(const GemmArgs &g, int dtype, cudaStream_t s);
@@ -126,6 +135,9 @@ struct AttnArgs {
   void *o; int ldo;
   const int *k_lens;      // device [B] or NULL
   float scale;
+  // optional per-query-row RMS factor folded into the logit scale:
+  // scale_row = scale / sqrt(sum_{t < q_ss_parts} q_ss[row * q_ss_stride + t] / q_ss_n + q_ss_eps)
+  const float *q_ss; int q_ss_stride; int q_ss_parts; float q_ss_n; float q_ss_eps;
 };
 int attention_simt(const AttnArgs &a, int dtype, cudaStream_t s);
 int attention_tc(const AttnArgs &a, cudaStream_t s);      // bf16, d = 128
@@ -147,6 +159,10 @@ int launch_rmsnorm_rope(void *p, int dtype, int rows, int ld, int D, int head_di
 // In place 3D RoPE only (no norm), rows of a [rows, heads*d] strided matrix.
 int launch_rope_only(void *p, int dtype, int rows, int ld, int D, int head_dim,
                      const float *rope, int rope_max_pos, int F, int H, int W, cudaStream_t s);
+// In place: row r of a strided bf16 matrix (D columns) *= 1/sqrt(S/D + eps),
+// S = sum of the `parts` partial sums at ss[r * ss_stride + 0 .. parts-1].
+int launch_scale_rows(void *p, int rows, int ld, int D, const float *ss, int ss_stride, int parts,
+                      float eps, cudaStream_t s);
 int launch_rope_table(int head_dim, int max_pos, double theta, float *table, cudaStream_t s);
 int launch_euler_cfg(float *x, const void *vc, const void *vu, int vdt, size_t n, float scale,
                      float dt, cudaStream_t s);

@@ -215,6 +215,45 @@ int launch_rope_only(void *p, int dtype, int rows, int ld, int D, int head_dim,
 }
 
 // ----------------------------------------------------------------------------
+// k rows of the tensor-core path: k[r] *= 1 / sqrt(ss[r] / D + eps) in place
+// (the QKV epilogue wrote gamma * RoPE(y) and the row's sum of squares of y).
+// One warp per row, 16-byte vectors.
+// ----------------------------------------------------------------------------
+__global__ void scale_rows_kernel(__nv_bfloat16 *__restrict__ p, int rows, int ld, int D,
+                                  const float *__restrict__ ss, int ss_stride, int parts, float inv_d,
+                                  float eps) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float part = lane < parts ? ss[(size_t)row * ss_stride + lane] : 0.f;
+  const float r = rsqrtf(warp_sum(part) * inv_d + eps);
+  uint4 *pr = reinterpret_cast<uint4 *>(p + (size_t)row * ld);
+  for (int c = lane; c < D / 8; c += 32) {
+    uint4 u = pr[c];
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162 *>(&w[e]);
+      float2 f = __bfloat1622float2(h);
+      h = __floats2bfloat162_rn(f.x * r, f.y * r);
+      w[e] = *reinterpret_cast<uint32_t *>(&h);
+    }
+    pr[c] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+int launch_scale_rows(void *p, int rows, int ld, int D, const float *ss, int ss_stride, int parts,
+                      float eps, cudaStream_t s) {
+  if (rows == 0) return WAN_OK;
+  if (D % 8 || ld % 8 || parts < 1 || parts > 32) return set_error(WAN_EUNSUPPORTED, "scale_rows: D=%d", D);
+  const int warps = 8;
+  scale_rows_kernel<<<(rows + warps - 1) / warps, warps * 32, 0, s>>>(
+      static_cast<__nv_bfloat16 *>(p), rows, ld, D, ss, ss_stride, parts, 1.0f / (float)D, eps);
+  WAN_CHECK_LAUNCH("scale_rows");
+  return WAN_OK;
+}
+
+// ----------------------------------------------------------------------------
 // RoPE table: one thread per (pos, pair). Angle in fp64, stored as fp32.
 // ----------------------------------------------------------------------------
 __global__ void rope_table_kernel(int half, int max_pos, double theta, float *__restrict__ table) {

@@ -121,6 +121,7 @@ int launch_t(const GemmArgs &g, cudaStream_t s) {
 }  // namespace
 
 int gemm_simt(const GemmArgs &g, int dtype, cudaStream_t s) {
+  if (g.epi == EPI_QKNORM) return set_error(WAN_EUNSUPPORTED, "gemm_simt: q/k-norm epilogue is tensor-core only");
   if (g.K % BK || g.N % 8 || g.segN % 8 || g.lda % 4)
     return set_error(WAN_EUNSUPPORTED, "gemm_simt: M=%d N=%d K=%d", g.M, g.N, g.K);
   if (g.M == 0 || g.N == 0) return WAN_OK;

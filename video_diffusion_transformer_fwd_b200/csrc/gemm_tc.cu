@@ -50,6 +50,9 @@ struct TcParams {
   void *C; int ldc;
   float *X; int ldx;
   const float *gate; int gate_stride; int rows_per_gate;
+  // q/k RMSNorm + RoPE epilogue (EPI_QKNORM)
+  const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
+  const float *rope; int rope_mask; int L, H, W; int head_dim;
   int *watchdog;
 };
 
@@ -214,6 +217,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int seg = n0 / p.segN;
       const __nv_bfloat16 *bias = static_cast<const __nv_bfloat16 *>(p.bias[seg]);
       const int nn0 = n0 - seg * p.segN;
+      // q/k RMSNorm + RoPE epilogue: per-row sum of squares of y, gamma, rotation
+      float sq = 0.f;
+      int ss_col = -1, tpos = 0, hpos = 0, wpos = 0;
+      bool do_rope = false;
+      const float *gam = nullptr;
+      if (EPI == EPI_QKNORM) {
+        ss_col = p.ss_col[seg];
+        gam = p.gamma[seg];
+        do_rope = (p.rope_mask >> seg) & 1;
+        const int tok = (m < p.M ? m : 0) % p.L;
+        tpos = tok / (p.H * p.W);
+        hpos = (tok / p.W) % p.H;
+        wpos = tok % p.W;
+      }
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -268,6 +285,35 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
           ++stg_count;
         } else {
+          if (EPI == EPI_QKNORM) {
+            const int col = nn0 + c * 32;            // column within the segment
+            if (ss_col >= 0) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sq = fmaf(v[j], v[j], sq);
+            }
+            if (gam) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 4) {
+                const float4 g4 = *reinterpret_cast<const float4 *>(gam + col + j);
+                v[j] *= g4.x; v[j + 1] *= g4.y; v[j + 2] *= g4.z; v[j + 3] *= g4.w;
+              }
+            }
+            if (do_rope) {
+              // pair jp of the head rotates with the t, h or w index:
+              // [c - 2(c/3), c/3, c/3] pairs, c = head_dim / 2
+              const int half = p.head_dim >> 1, c3 = half / 3, pt = half - 2 * c3;
+              const int jp0 = (col % p.head_dim) >> 1;
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int jp = jp0 + e;
+                const int pos = jp < pt ? tpos : (jp < pt + c3 ? hpos : wpos);
+                const float2 cs = *reinterpret_cast<const float2 *>(p.rope + ((size_t)pos * half + jp) * 2);
+                const float x0 = v[2 * e], x1 = v[2 * e + 1];
+                v[2 * e] = x0 * cs.x - x1 * cs.y;
+                v[2 * e + 1] = x0 * cs.y + x1 * cs.x;
+              }
+            }
+          }
           __nv_bfloat16 *cr = static_cast<__nv_bfloat16 *>(p.C) + (size_t)m * p.ldc + n;
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
@@ -287,6 +333,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
         }
       }
+      // one partial sum per (row, column tile of the segment): no atomics
+      if (EPI == EPI_QKNORM && ss_col >= 0 && m < p.M)
+        p.ss[(size_t)m * p.ss_stride + ss_col * (p.segN / BN) + nn0 / BN] = sq;
     }
   }
 
@@ -341,6 +390,14 @@ bool gemm_tc_supported(const GemmArgs &g) {
   if (g.lda % 8) return false;
   if (g.epi != EPI_RESID && g.ldc % 8) return false;
   if (g.epi == EPI_RESID && (g.ldx % 4 || !aligned16(g.X) || (g.gate && g.gate_stride % 4))) return false;
+  if (g.epi == EPI_QKNORM) {
+    for (int i = 0; i < g.nseg; ++i) {
+      if (g.ss_col[i] >= 0 && !g.ss) return false;
+      if (g.gamma[i] && !aligned16(g.gamma[i])) return false;
+    }
+    if (g.rope && (g.head_dim % 32 || g.segN % g.head_dim)) return false;
+    if (g.segN % BN) return false;             // whole column tiles per segment (partial sums)
+  }
   for (int i = 0; i < g.nseg; ++i)
     if (!aligned16(g.Bseg[i]) || (g.bias[i] && !aligned16(g.bias[i]))) return false;
   return aligned16(g.A);
@@ -364,12 +421,21 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   for (int i = 0; i < 3; ++i) p.bias[i] = i < g.nseg ? g.bias[i] : nullptr;
   p.C = g.C; p.ldc = g.ldc; p.X = g.X; p.ldx = g.ldx;
   p.gate = g.gate; p.gate_stride = g.gate_stride; p.rows_per_gate = g.rows_per_gate > 0 ? g.rows_per_gate : 1;
+  for (int i = 0; i < 3; ++i) {
+    p.gamma[i] = i < g.nseg ? g.gamma[i] : nullptr;
+    p.ss_col[i] = i < g.nseg ? g.ss_col[i] : -1;
+  }
+  p.ss = g.ss; p.ss_stride = g.ss_stride;
+  p.rope = g.rope; p.rope_mask = g.rope ? g.rope_mask : 0;
+  p.L = g.F * g.H * g.W > 0 ? g.F * g.H * g.W : 1; p.H = g.H > 0 ? g.H : 1; p.W = g.W > 0 ? g.W : 1;
+  p.head_dim = g.head_dim > 0 ? g.head_dim : 128;
   p.watchdog = watchdog_ptr();
   CUtensorMap tx = ta;
   if (g.epi == EPI_RESID && (rc = encode_tmap_2d_f32(&tx, g.X, g.N, g.M, (uint64_t)g.ldx * 4, 32, 32))) return rc;
   switch (g.epi) {
     case EPI_STORE: return launch<EPI_STORE>(ta, tb, tx, p, s);
     case EPI_GELU: return launch<EPI_GELU>(ta, tb, tx, p, s);
+    case EPI_QKNORM: return launch<EPI_QKNORM>(ta, tb, tx, p, s);
     default: return launch<EPI_RESID>(ta, tb, tx, p, s);
   }
 }
