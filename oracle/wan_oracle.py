@@ -378,3 +378,122 @@ def denoise_step(x_tokens, ctx_cond, ctx_uncond, ctx_lens, e0, blocks, heads, gr
     for w in blocks:
         xb = block_forward(xb, ctx, ctx_lens, e, w, heads, grid, eps, theta)
     return euler_cfg_step(x_tokens, xb[0], xb[1], guide_scale, sigma, sigma_next)
+
+
+# --------------------------------------------------------------------------
+# Whole-model step on latents ([WALK] structure, forward and time-projection
+# snippets, MoE expert-switch and sampling-loop snippets; [DIFFUSERS]
+# "3D Patchify" and "Unpatchify"; [TRACE] section 4 "DIT").
+#
+# Readings taken where the pages are silent:
+# * freq_dim = 256 and the sinusoidal embedding of t is [cos(t w_j), sin(t w_j)],
+#   w_j = 10000^(-j / (freq_dim/2)), j < freq_dim/2.
+# * The head (``Head(dim, out_dim, patch_size, eps)`` called as head(x, e))
+#   is LayerNorm without affine, modulated like the block's AdaLN by two
+#   chunks (shift, scale) of (head_modulation + e), then Linear(dim ->
+#   out_dim * 1*2*2); e is the time embedding before the 6 x dim projection.
+# * Patch embedding weight [dim, C, 1, 2, 2] (Conv3d); a token's input
+#   features are ordered (c, kt, kh, kw) like the flattened weight.
+# * The head's out_dim*4 features of a token are ordered (kt, kh, kw, c),
+#   channel fastest, when folded back into [C, F, 2H, 2W].
+# * The denoiser is called at timestep t = 1000 * sigma.
+# --------------------------------------------------------------------------
+
+MODEL_WEIGHT_NAMES = ("patch_w", "patch_b", "text_w1", "text_b1", "text_w2", "text_b2",
+                      "time_w1", "time_b1", "time_w2", "time_b2", "proj_w", "proj_b",
+                      "head_mod", "head_w", "head_b")
+
+
+def sinusoidal_embedding(freq_dim: int, t) -> np.ndarray:
+    """[B, freq_dim]: cos then sin of t * 10000^(-j/half), j < half."""
+    t = np.asarray(t, F64).reshape(-1)
+    half = freq_dim // 2
+    w = 10000.0 ** (-np.arange(half, dtype=F64) / half)
+    a = t[:, None] * w[None, :]
+    return np.concatenate([np.cos(a), np.sin(a)], axis=1)
+
+
+def silu(z):
+    z = np.asarray(z, F64)
+    return z / (1.0 + np.exp(-z))
+
+
+def time_embed(t, mw, freq_dim=256):
+    """e = Linear(SiLU(Linear(sinusoid(t)))) and e0 = Linear(SiLU(e)) as
+    [B, 6, dim] ([WALK] structure and time-projection snippets)."""
+    s = sinusoidal_embedding(freq_dim, t)
+    e = linear(silu(linear(s, mw["time_w1"], mw["time_b1"])), mw["time_w2"], mw["time_b2"])
+    e0 = linear(silu(e), mw["proj_w"], mw["proj_b"])
+    return e, e0.reshape(e.shape[0], 6, -1)
+
+
+def text_embed(ctx_raw, mw):
+    """Linear(4096 -> dim), GELU-tanh, Linear(dim -> dim) per text token."""
+    return linear(gelu_tanh(linear(ctx_raw, mw["text_w1"], mw["text_b1"])), mw["text_w2"], mw["text_b2"])
+
+
+def patchify(latent):
+    """[B, C, F, H, W] -> tokens [B, F*(H/2)*(W/2), C*4], token order (f, h, w),
+    features (c, kh, kw) with kt = 0 (the (1, 2, 2) Conv3d's receptive field)."""
+    x = np.asarray(latent, F64)
+    B, C, F, H, W = x.shape
+    x = x.reshape(B, C, F, H // 2, 2, W // 2, 2)          # b c f h kh w kw
+    x = x.transpose(0, 2, 3, 5, 1, 4, 6)                  # b f h w c kh kw
+    return x.reshape(B, F * (H // 2) * (W // 2), C * 4)
+
+
+def patch_embed(latent, mw):
+    """Conv3d(C, dim, kernel (1,2,2), stride (1,2,2)) flattened to tokens."""
+    dim = np.asarray(mw["patch_w"]).shape[0]
+    return linear(patchify(latent), np.asarray(mw["patch_w"], F64).reshape(dim, -1), mw["patch_b"])
+
+
+def head(x, e, mw, eps):
+    """LN(x) (1 + m1) + m0 with m = head_modulation + e, then Linear."""
+    m = np.asarray(mw["head_mod"], F64)[None] + np.asarray(e, F64)[:, None, :]   # [B, 2, dim]
+    u = layer_norm(x, eps) * (1.0 + m[:, 1, None, :]) + m[:, 0, None, :]
+    return linear(u, mw["head_w"], mw["head_b"])
+
+
+def unpatchify(tokens, grid, channels):
+    """tokens [B, L, 4*C] (features (kt, kh, kw, c)) -> [B, C, F, 2H, 2W]."""
+    F, H, W = grid
+    t = np.asarray(tokens, F64)
+    B = t.shape[0]
+    t = t.reshape(B, F, H, W, 1, 2, 2, channels)           # b f h w kt kh kw c
+    t = t.transpose(0, 7, 1, 4, 2, 5, 3, 6)                # b c f kt h kh w kw
+    return t.reshape(B, channels, F, 2 * H, 2 * W)
+
+
+def model_forward(latent, t, ctx_raw, ctx_lens, mw, blocks, heads, eps, theta=1e4, freq_dim=256):
+    """WanModel forward on latents ([WALK] forward snippet): patch embedding,
+    flatten, time and text embeddings, the block stack, head, unpatchify."""
+    latent = np.asarray(latent, F64)
+    B, C, Fl, Hl, Wl = latent.shape
+    grid = (Fl, Hl // 2, Wl // 2)
+    x = patch_embed(latent, mw)
+    e, e0 = time_embed(t, mw, freq_dim)
+    ctx = text_embed(ctx_raw, mw)
+    for w in blocks:
+        x = block_forward(x, ctx, ctx_lens, e0, w, heads, grid, eps, theta)
+    out_c = np.asarray(mw["head_w"]).shape[0] // 4
+    return unpatchify(head(x, e, mw, eps), grid, out_c)
+
+
+def select_expert(t: float, boundary: float) -> str:
+    """Two-expert switch ([WALK] MoE snippet): the high-noise model when
+    t >= boundary (boundary = 0.875 * 1000 for T2V, 900 for I2V)."""
+    return "high" if t >= boundary else "low"
+
+
+def model_denoise_step(latent, sigma, sigma_next, ctx_cond, ctx_uncond, mw, blocks, heads, eps,
+                       guide_scale, theta=1e4, freq_dim=256):
+    """One CFG flow-matching Euler step on the latent: the model runs on the
+    same latent at t = 1000 sigma for both contexts, v = v_u + s (v_c - v_u),
+    latent + (sigma' - sigma) v."""
+    latent = np.asarray(latent, F64)
+    lat2 = np.stack([latent, latent])
+    ctx = np.stack([np.asarray(ctx_cond, F64), np.asarray(ctx_uncond, F64)])
+    t = np.array([1000.0 * sigma] * 2)
+    v = model_forward(lat2, t, ctx, None, mw, blocks, heads, eps, theta, freq_dim)
+    return euler_cfg_step(latent, v[0], v[1], guide_scale, sigma, sigma_next)
