@@ -175,6 +175,66 @@ int wan_block_forward_noalloc(const wan_dims *dims, int B, float *x, const void 
                               const wan_block_weights *w, const float *rope,
                               int rope_max_pos, wan_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Whole-model forward on latents ([WALK] WanModel structure and forward
+ * snippets, time-projection snippet; [DIFFUSERS] "3D Patchify", "Unpatchify").
+ *   x   = Conv3d(C_in, dim, kernel = stride = (1,2,2))(latent), flattened to
+ *         tokens (t, h, w order)
+ *   e   = Linear(SiLU(Linear(sinusoid(t))))  (freq_dim features: cos | sin of
+ *         t * 10000^(-j/(freq_dim/2)))
+ *   e0  = Linear(SiLU(e)) as [B, 6, dim]
+ *   ctx = Linear(GELU_tanh(Linear(text)))   (text_dim -> dim -> dim)
+ *   x   = blocks[0..n-1](x, ctx, e0)        (wan_block_forward)
+ *   y   = Linear(LN(x) (1 + m1) + m0), m = head_modulation + e  (C_out * 4 outputs)
+ *   out = y folded back to [C_out, F, H, W] (token features ordered
+ *         (kt, kh, kw, c), channel fastest)
+ * ------------------------------------------------------------------------- */
+typedef struct {
+  int C_in, C_out;      /* latent channels in / out (16 / 16 for T2V)           */
+  int F, H, W;          /* latent grid before patching; H and W even; the token
+                           grid is (F, H/2, W/2)                                 */
+  int dim, heads, ffn_dim;
+  int text_len;         /* T text tokens per sequence                            */
+  int text_dim;         /* width of the text encoder features (4096 for umT5)   */
+  int freq_dim;         /* sinusoidal time features (256)                        */
+  float eps;
+  int dtype;            /* WAN_F32 | WAN_BF16, as in wan_dims                    */
+} wan_model_dims;
+
+/* (dt) = wan_model_dims.dtype; others float32. */
+typedef struct {
+  const void *patch_w, *patch_b;      /* (dt) [dim, C_in*4] (Conv3d weight [dim, C_in, 1, 2, 2]), [dim] */
+  const void *text_w1, *text_b1;      /* (dt) [dim, text_dim], [dim]           */
+  const void *text_w2, *text_b2;      /* (dt) [dim, dim], [dim]                */
+  const float *time_w1, *time_b1;     /* [dim, freq_dim], [dim]                */
+  const float *time_w2, *time_b2;     /* [dim, dim], [dim]                     */
+  const float *proj_w, *proj_b;       /* [6*dim, dim], [6*dim]                 */
+  const float *head_mod;              /* [2, dim] (shift, scale) bias           */
+  const void *head_w, *head_b;        /* (dt) [C_out*4, dim], [C_out*4]        */
+} wan_model_weights;
+
+/* Workspace bytes for wan_model_forward (0 on invalid dims). */
+size_t wan_model_workspace_bytes(const wan_model_dims *dims, int B);
+
+/* wan_model_forward -- the model above for B sequences.
+ *   latent  float32 [B, C_in, F, H, W]; t float32 [B] (device) timesteps.
+ *   text    (dt) [B, T, text_dim] text encoder features; ctx_lens as in
+ *           wan_block_forward (device int32 [B] or NULL).
+ *   w       model weights; blocks: HOST array of num_blocks block weights.
+ *   rope    table from wan_rope_freqs(dim/heads, rope_max_pos >= the token grid).
+ *   out     float32 [B, C_out, F, H, W] (the predicted velocity).
+ * Constraints: wan_dims rules for the token grid (F, H/2, W/2) and dim / heads /
+ * ffn_dim; H, W even; C_in * 4 and freq_dim multiples of 8; text_dim a multiple
+ * of 64 (when text_len > 0); num_blocks >= 0; every pointer 16-byte aligned.
+ * The workspace holds the token stream, the embeddings and one block
+ * workspace; the head's normalised tokens reuse the block's ACT buffer.
+ * Errors: as wan_block_forward. */
+int wan_model_forward(const wan_model_dims *dims, int B, const float *latent, const float *t,
+                      const void *text, const int *ctx_lens, const wan_model_weights *w,
+                      const wan_block_weights *blocks, int num_blocks, const float *rope,
+                      int rope_max_pos, float *out, void *workspace, size_t ws_bytes,
+                      wan_stream_t stream);
+
 /* wan_attention -- softmax attention, non-causal, every head
  * ([WALK] self-attention snippet: global window, key lengths).
  *   B, heads, Lq, Lk, head_dim   sizes (head_dim 128 for WAN_BF16; 32, 64
@@ -238,7 +298,8 @@ int wan_selftest_watchdog(wan_stream_t stream);
 #define WAN_K_EULER        7  /* CFG + Euler update                           */
 #define WAN_K_MISC         8  /* modulation combine, RoPE table               */
 #define WAN_K_ATTN_TC      9  /* tensor-core attention via wan_attention      */
-#define WAN_K_COUNT       10
+#define WAN_K_MODEL       10  /* patchify, embeddings, head, unpatchify       */
+#define WAN_K_COUNT       11
 int wan_profile_enable(int on);
 int wan_profile_read(int kernel_class, int *launches, double *total_ms);
 

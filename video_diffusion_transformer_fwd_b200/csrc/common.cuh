@@ -93,13 +93,14 @@ inline size_t dtype_size(int dt) { return dt == WAN_BF16 ? 2 : 4; }
 
 // ---------------------------------------------------------------- internal kernels API
 
-enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_QKNORM = 3 };
+enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_QKNORM = 3, EPI_SILU = 4 };
 
 // C = A B^T (+ bias) with a fused epilogue. A [M,K] row-major (lda),
 // B given as up to 3 row-major segments [segN, K] (ldb = K) stacked along N,
 // so one call can multiply by [Wq; Wk; Wv]. bias per segment [segN] (or NULL).
 //   EPI_STORE: C[m,n] = acc + bias
 //   EPI_GELU:  C[m,n] = gelu_tanh(acc + bias)
+//   EPI_SILU:  C[m,n] = silu(acc + bias)          (CUDA-core GEMM only)
 //   EPI_RESID: X[m,n] += g * (acc + bias), g = gate[(m / rows_per_gate) *
 //              gate_stride + n] or 1 when gate == NULL  (X float32, ldx)
 //   EPI_QKNORM (tensor-core path): per segment s, y = acc + bias; when

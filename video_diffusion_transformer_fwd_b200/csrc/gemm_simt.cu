@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(THREADS) gemm_simt_kernel(const GemmArgs g) {
     for (int j = 0; j < 8; ++j) {
       v[j] = acc[i][j] + bias[j];
       if (EPI == EPI_GELU) v[j] = gelu_tanh(v[j]);
+      if (EPI == EPI_SILU) v[j] = v[j] / (1.0f + expf(-v[j]));
     }
     if (EPI == EPI_RESID) {
       float *xr = g.X + (size_t)m * g.ldx + nb;
@@ -113,6 +114,7 @@ int launch_t(const GemmArgs &g, cudaStream_t s) {
   switch (g.epi) {
     case EPI_STORE: gemm_simt_kernel<T, EPI_STORE><<<grid, THREADS, 0, s>>>(g); break;
     case EPI_GELU: gemm_simt_kernel<T, EPI_GELU><<<grid, THREADS, 0, s>>>(g); break;
+    case EPI_SILU: gemm_simt_kernel<T, EPI_SILU><<<grid, THREADS, 0, s>>>(g); break;
     default: gemm_simt_kernel<T, EPI_RESID><<<grid, THREADS, 0, s>>>(g); break;
   }
   WAN_CHECK_LAUNCH("gemm_simt");

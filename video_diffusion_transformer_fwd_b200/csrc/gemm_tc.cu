@@ -384,6 +384,7 @@ int launch(const CUtensorMap &ta, const CUtensorMap *tb, const CUtensorMap &tx, 
 }  // namespace
 
 bool gemm_tc_supported(const GemmArgs &g) {
+  if (g.epi == EPI_SILU) return false;
   if (g.M < 1 || g.N < 32 || g.K < BK || g.K % BK || g.N % 32) return false;
   if (g.nseg < 1 || g.nseg > 3 || g.segN * g.nseg != g.N) return false;
   if (g.nseg > 1 && g.segN % BN) return false;

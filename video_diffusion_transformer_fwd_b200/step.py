@@ -51,3 +51,55 @@ class DenoiseStep:
                                          c.guide_scale, c.sigma, c.sigma_next,
                                          wan._stream(stream)))
         return self.x
+
+
+class ModelDenoiseStep:
+    """One CFG flow-matching Euler step on the latent through the whole model
+    (wan_model_forward on the CFG pair at t = 1000 sigma, then
+    wan_euler_cfg_step on the latent). With two experts, the high-noise one
+    runs while t >= boundary ("Wan2.2 code walkthrough" (newtid.com), MoE
+    snippet: boundary 0.875 * 1000 for text-to-video, 900 for image-to-video).
+
+    ``experts`` maps "high" / "low" to (model weight dict, list of block weight
+    dicts); a single expert may be passed as {"high": ...} with boundary 0.
+    """
+
+    def __init__(self, dims: "wan.wan_model_dims", experts: dict, text, latent,
+                 boundary: float = 875.0, ctx_lens=None, rope_max_pos: int = 1024,
+                 theta: float = 1e4, device: str = "cuda"):
+        self.dims = dims
+        self.boundary = boundary
+        self.experts = {k: (wan.make_model_weights(mw), wan.make_block_array(bl))
+                        for k, (mw, bl) in experts.items()}
+        self._keep = experts                         # device tensors stay alive
+        self.text = text                             # [2, T, text_dim]: cond, uncond
+        self.ctx_lens = ctx_lens
+        self.latent = latent                         # [C_in, F, H, W] float32, the state
+        head_dim = dims.dim // dims.heads
+        self.rope = wan.rope_freqs(head_dim, rope_max_pos, theta, device=device)
+        self.lat2 = torch.empty((2,) + tuple(latent.shape), dtype=torch.float32, device=device)
+        self.t = torch.empty(2, dtype=torch.float32, device=device)
+        self.v = torch.empty((2, dims.C_out, dims.F, dims.H, dims.W), dtype=torch.float32,
+                             device=device)
+        self.ws = wan.alloc_model_workspace(dims, 2, device=device)
+
+    def expert(self, sigma: float) -> str:
+        t = 1000.0 * sigma
+        if "low" not in self.experts or t >= self.boundary:
+            return "high"
+        return "low"
+
+    def step(self, sigma: float, sigma_next: float, guide_scale: float, stream=None):
+        s = wan._stream(stream)
+        mw, blocks = self.experts[self.expert(sigma)]
+        self.lat2[0].copy_(self.latent)
+        self.lat2[1].copy_(self.latent)
+        self.t.fill_(1000.0 * sigma)
+        wan.check(wan.wan_model_forward(self.dims, 2, self.lat2.data_ptr(), self.t.data_ptr(),
+                                        wan._ptr(self.text), wan._ptr(self.ctx_lens), mw, blocks,
+                                        len(blocks), self.rope.data_ptr(), self.rope.shape[0],
+                                        self.v.data_ptr(), self.ws.data_ptr(), self.ws.numel(), s))
+        wan.check(wan.wan_euler_cfg_step(self.latent.data_ptr(), self.v[0].data_ptr(),
+                                         self.v[1].data_ptr(), wan.WAN_F32, self.latent.numel(),
+                                         guide_scale, sigma, sigma_next, s))
+        return self.latent

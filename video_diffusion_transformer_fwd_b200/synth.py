@@ -102,6 +102,47 @@ def step_weights(cfg, device="cpu", seed=0):
             for i in range(cfg.blocks)]
 
 
+MODEL_WEIGHT_SPECS = (
+    # name, shape key, is_matrix_dtype (False: float32)
+    ("patch_w", "D,4C", True), ("patch_b", "D", True),
+    ("text_w1", "D,TD", True), ("text_b1", "D", True),
+    ("text_w2", "D,D", True), ("text_b2", "D", True),
+    ("time_w1", "D,FD", False), ("time_b1", "D", False),
+    ("time_w2", "D,D", False), ("time_b2", "D", False),
+    ("proj_w", "6D,D", False), ("proj_b", "6D", False),
+    ("head_mod", "2,D", False),
+    ("head_w", "4CO,D", True), ("head_b", "4CO", True),
+)
+
+
+def model_weights(C_in, C_out, dim, text_dim, freq_dim=256, dtype="bf16", device="cpu",
+                  seed=50000, std=0.02, head_mod_std=0.1):
+    """The embeddings and head around the block stack (all N(0, std) except
+    head_mod, N(0, head_mod_std)). The patch weight is the Conv3d weight
+    [dim, C_in, 1, 2, 2] flattened to [dim, C_in * 4]."""
+    tdt = TORCH_DTYPES[dtype]
+    sizes = {"D": dim, "4C": 4 * C_in, "TD": text_dim, "FD": freq_dim, "6D": 6 * dim, "2": 2,
+             "4CO": 4 * C_out}
+    out = {}
+    for idx, (name, key, is_mat) in enumerate(MODEL_WEIGHT_SPECS):
+        shape = tuple(sizes[k] for k in key.split(","))
+        t = _normal(shape, seed + idx, device, head_mod_std if name == "head_mod" else std)
+        out[name] = t.to(tdt).contiguous() if is_mat else t.contiguous()
+    return out
+
+
+def model_inputs(B, C_in, F, H, W, text_len, text_dim, dtype="bf16", device="cpu", seed=60000,
+                 same_latent=False):
+    """latent [B, C_in, F, H, W] float32 N(0, 1) (``same_latent``: sequence 0
+    repeated, the CFG pair), text features [B, text_len, text_dim] N(0, 1) in
+    ``dtype``."""
+    tdt = TORCH_DTYPES[dtype]
+    nb = 1 if same_latent else B
+    lat = _normal((nb, C_in, F, H, W), seed, device, 1.0).expand(B, C_in, F, H, W).contiguous()
+    text = _normal((B, text_len, text_dim), seed + 1, device, 1.0).to(tdt).contiguous()
+    return {"latent": lat, "text": text}
+
+
 def attention_inputs(B, Lq, Lk, heads, head_dim, dtype="bf16", device="cpu", seed=500,
                      std=1.0):
     """q [B, Lq, n, d], k and v [B, Lk, n, d] in ``dtype``."""

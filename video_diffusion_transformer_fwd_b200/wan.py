@@ -20,10 +20,10 @@ WAN_NOALLOC_WORKSPACE_BYTES = 16 << 20
 (WAN_WS_ACT, WAN_WS_QKV, WAN_WS_O, WAN_WS_QC, WAN_WS_KVC, WAN_WS_OC, WAN_WS_H, WAN_WS_MOD,
  WAN_WS_STATS) = range(9)
 (WAN_K_GEMM_TC, WAN_K_GEMM_SIMT, WAN_K_ATTN_SELF, WAN_K_ATTN_CROSS, WAN_K_ATTN_SIMT, WAN_K_LAYERNORM,
- WAN_K_QKNORM_ROPE, WAN_K_EULER, WAN_K_MISC, WAN_K_ATTN_TC) = range(10)
-WAN_K_COUNT = 10
+ WAN_K_QKNORM_ROPE, WAN_K_EULER, WAN_K_MISC, WAN_K_ATTN_TC, WAN_K_MODEL) = range(11)
+WAN_K_COUNT = 11
 KERNEL_CLASS_NAMES = ("gemm_tc", "gemm_simt", "attn_self", "attn_cross", "attn_simt", "layernorm",
-                      "qknorm_rope", "euler_cfg", "misc", "attn_tc")
+                      "qknorm_rope", "euler_cfg", "misc", "attn_tc", "model")
 STATUS_NAMES = {0: "WAN_OK", -1: "WAN_EINVAL", -2: "WAN_EALIGN", -3: "WAN_EUNSUPPORTED",
                 -4: "WAN_ECUDA", -5: "WAN_ETIMEOUT"}
 
@@ -49,6 +49,23 @@ class wan_block_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
 
 
+class wan_model_dims(ctypes.Structure):
+    _fields_ = [("C_in", ctypes.c_int), ("C_out", ctypes.c_int), ("F", ctypes.c_int),
+                ("H", ctypes.c_int), ("W", ctypes.c_int), ("dim", ctypes.c_int),
+                ("heads", ctypes.c_int), ("ffn_dim", ctypes.c_int), ("text_len", ctypes.c_int),
+                ("text_dim", ctypes.c_int), ("freq_dim", ctypes.c_int), ("eps", ctypes.c_float),
+                ("dtype", ctypes.c_int)]
+
+
+MODEL_WEIGHT_FIELDS = ("patch_w", "patch_b", "text_w1", "text_b1", "text_w2", "text_b2",
+                       "time_w1", "time_b1", "time_w2", "time_b2", "proj_w", "proj_b",
+                       "head_mod", "head_w", "head_b")
+
+
+class wan_model_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in MODEL_WEIGHT_FIELDS]
+
+
 _c_int, _vp, _sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t
 
 _SIGS = {
@@ -68,6 +85,11 @@ _SIGS = {
     "wan_profile_enable": (_c_int, [_c_int]),
     "wan_selftest_watchdog": (_c_int, [_vp]),
     "wan_profile_read": (_c_int, [_c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]),
+    "wan_model_workspace_bytes": (_sz, [ctypes.POINTER(wan_model_dims), _c_int]),
+    "wan_model_forward": (_c_int, [ctypes.POINTER(wan_model_dims), _c_int, _vp, _vp, _vp, _vp,
+                                   ctypes.POINTER(wan_model_weights),
+                                   ctypes.POINTER(wan_block_weights), _c_int, _vp, _c_int, _vp,
+                                   _vp, _sz, _vp]),
 }
 
 _lib = None
@@ -138,6 +160,17 @@ def wan_attention(B, heads, Lq, Lk, head_dim, dtype, q, k, v, o, k_lens, scale, 
 def wan_euler_cfg_step(x, v_cond, v_uncond, v_dtype, n, guide_scale, sigma, sigma_next, stream):
     return load().wan_euler_cfg_step(x, v_cond, v_uncond, v_dtype, n, guide_scale, sigma,
                                      sigma_next, stream)
+
+
+def wan_model_workspace_bytes(dims, B):
+    return load().wan_model_workspace_bytes(ctypes.byref(dims), B)
+
+
+def wan_model_forward(dims, B, latent, t, text, ctx_lens, weights, blocks, num_blocks, rope,
+                      rope_max_pos, out, workspace, ws_bytes, stream):
+    return load().wan_model_forward(ctypes.byref(dims), B, latent, t, text, ctx_lens,
+                                    ctypes.byref(weights), blocks, num_blocks, rope, rope_max_pos,
+                                    out, workspace, ws_bytes, stream)
 
 
 def wan_device_status(stream):
@@ -276,3 +309,53 @@ def euler_cfg_step(x, v_cond, v_uncond, guide_scale, sigma, sigma_next, stream=N
 
 def device_status(stream=None) -> int:
     return wan_device_status(_stream(stream))
+
+
+def make_model_dims(C_in, C_out, F, H, W, dim, heads, ffn_dim, text_len, text_dim, freq_dim=256,
+                    eps=1e-6, dtype="bf16") -> wan_model_dims:
+    code = {"bf16": WAN_BF16, "f32": WAN_F32}[dtype] if isinstance(dtype, str) else int(dtype)
+    return wan_model_dims(C_in, C_out, F, H, W, dim, heads, ffn_dim, text_len, text_dim, freq_dim,
+                          eps, code)
+
+
+def make_model_weights(w: dict) -> wan_model_weights:
+    for n in MODEL_WEIGHT_FIELDS:
+        if w.get(n) is not None and not w[n].is_contiguous():
+            raise ValueError(f"weight {n} must be contiguous")
+    return wan_model_weights(*[_ptr(w.get(n)) for n in MODEL_WEIGHT_FIELDS])
+
+
+def make_block_array(blocks) -> ctypes.Array:
+    """A C array of wan_block_weights from a list of weight dicts (or structs)."""
+    arr = (wan_block_weights * len(blocks))()
+    for i, b in enumerate(blocks):
+        arr[i] = b if isinstance(b, wan_block_weights) else make_weights(b)
+    return arr
+
+
+def alloc_model_workspace(dims: wan_model_dims, B: int, device="cuda"):
+    torch = _torch()
+    n = wan_model_workspace_bytes(dims, B)
+    if n == 0:
+        raise WanError(WAN_EINVAL, last_error())
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def model_forward(dims: wan_model_dims, latent, t, text, weights, blocks, rope, workspace,
+                  ctx_lens=None, out=None, stream=None):
+    """Velocity of the whole model: latent [B, C_in, F, H, W] float32, t [B]
+    float32 timesteps (device), text [B, text_len, text_dim] in the compute
+    dtype. ``blocks`` is a list of block weight dicts or a make_block_array()
+    result. Returns out [B, C_out, F, H, W] float32."""
+    torch = _torch()
+    B = latent.shape[0]
+    if out is None:
+        out = torch.empty((B, dims.C_out, dims.F, dims.H, dims.W), dtype=torch.float32,
+                          device=latent.device)
+    mw = weights if isinstance(weights, wan_model_weights) else make_model_weights(weights)
+    arr = blocks if isinstance(blocks, ctypes.Array) else make_block_array(blocks)
+    check(wan_model_forward(dims, B, latent.data_ptr(), t.data_ptr(), _ptr(text), _ptr(ctx_lens),
+                            mw, arr, len(arr), rope.data_ptr(), rope.shape[0],
+                            out.data_ptr(), workspace.data_ptr(),
+                            workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
