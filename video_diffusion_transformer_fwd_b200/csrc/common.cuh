@@ -118,6 +118,7 @@ struct GemmArgs {
   void *C; int ldc;
   float *X; int ldx;
   const float *gate; int gate_stride; int rows_per_gate;
+  int x_store;            // EPI_RESID: x = g * y (overwrite) instead of x += g * y
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
   const float *rope; int rope_mask; int F, H, W; int head_dim;
 };
@@ -125,6 +126,9 @@ struct GemmArgs {
 int gemm_simt(const GemmArgs &g, int dtype, cudaStream_t s);
 int gemm_tc(const GemmArgs &g, cudaStream_t s);           // bf16 tcgen05 path
 bool gemm_tc_supported(const GemmArgs &g);
+// M <= 8 rows, one weight segment, STORE or SILU epilogue (gemv.cu)
+int gemm_smallm(const GemmArgs &g, int dtype, cudaStream_t s);
+bool gemm_smallm_supported(const GemmArgs &g);
 
 // Attention over rows of strided matrices. Sequence b, row r of q is at
 // q + (b*Lq + r)*ldq + head*d (likewise k, v with Lk, o with Lq).

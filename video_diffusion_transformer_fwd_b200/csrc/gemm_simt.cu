@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(THREADS) gemm_simt_kernel(const GemmArgs g) {
       const float *gr = g.gate ? g.gate + (size_t)(m / g.rows_per_gate) * g.gate_stride + nb : nullptr;
 #pragma unroll
       for (int j = 0; j < 8; j += 4) {
-        float4 xv = load4(xr + j);
+        float4 xv = g.x_store ? make_float4(0.f, 0.f, 0.f, 0.f) : load4(xr + j);
         float4 gv = gr ? load4(gr + j) : make_float4(1.f, 1.f, 1.f, 1.f);
         xv.x = fmaf(gv.x, v[j + 0], xv.x);
         xv.y = fmaf(gv.y, v[j + 1], xv.y);

@@ -15,7 +15,8 @@
 //   warps 2..5  epilogue in both CTAs: tcgen05.ld of this CTA's 128 rows
 //               (warp w reads TMEM lanes 32*(w%4)..+31), bias, GELU or gated
 //               residual, stores to global (the residual add x += g*y goes
-//               through a swizzled smem tile and a TMA reduce-add into x);
+//               through a swizzled smem tile and a TMA reduce-add into x,
+//               or a TMA store when x is written rather than accumulated);
 //               then a release arrive on the leader's "accumulator empty"
 //               barrier.
 // Tiles are walked in groups of 8 M-tiles (2048 rows) so a wave of pairs
@@ -49,7 +50,7 @@ struct TcParams {
   const void *bias[3];
   void *C; int ldc;
   float *X; int ldx;
-  const float *gate; int gate_stride; int rows_per_gate;
+  const float *gate; int gate_stride; int rows_per_gate; int x_store;
   // q/k RMSNorm + RoPE epilogue (EPI_QKNORM)
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
   const float *rope; int rope_mask; int L, H, W; int head_dim;
@@ -280,7 +281,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_reduce_add_2d(&tmX, smem_u32(buf), n, m0w);
+            if (p.x_store)
+              tma_store_2d(&tmX, smem_u32(buf), n, m0w);
+            else
+              tma_reduce_add_2d(&tmX, smem_u32(buf), n, m0w);
             bulk_commit_group();
           }
           ++stg_count;
@@ -422,6 +426,7 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   for (int i = 0; i < 3; ++i) p.bias[i] = i < g.nseg ? g.bias[i] : nullptr;
   p.C = g.C; p.ldc = g.ldc; p.X = g.X; p.ldx = g.ldx;
   p.gate = g.gate; p.gate_stride = g.gate_stride; p.rows_per_gate = g.rows_per_gate > 0 ? g.rows_per_gate : 1;
+  p.x_store = g.x_store;
   for (int i = 0; i < 3; ++i) {
     p.gamma[i] = i < g.nseg ? g.gamma[i] : nullptr;
     p.ss_col[i] = i < g.nseg ? g.ss_col[i] : -1;

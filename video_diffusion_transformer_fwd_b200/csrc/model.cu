@@ -142,6 +142,7 @@ ModelLayout model_layout(const wan_model_dims &m, int B) {
 }
 
 int gemm_any(const GemmArgs &g, int dtype, cudaStream_t s) {
+  if (gemm_smallm_supported(g)) return WAN_PROF(WAN_K_MODEL, s, gemm_smallm(g, dtype, s));
   if (dtype == WAN_BF16 && gemm_tc_supported(g)) return WAN_PROF(WAN_K_GEMM_TC, s, gemm_tc(g, s));
   return WAN_PROF(WAN_K_GEMM_SIMT, s, gemm_simt(g, dtype, s));
 }
@@ -205,7 +206,7 @@ int wan_model_forward(const wan_model_dims *dims, int B, const float *latent, co
   const wan_dims tok = token_dims(m);
   void *act = bws + wan_block_workspace_offset(&tok, B, WAN_WS_ACT);
 
-  // patch embedding: x = patches W^T + b, written into a zeroed fp32 stream
+  // patch embedding: x = patches W^T + b, stored as the fp32 token stream
   {
     const size_t n = (size_t)BL * m.C_in * 4;
     if (dt == WAN_BF16)
@@ -215,11 +216,11 @@ int wan_model_forward(const wan_model_dims *dims, int B, const float *latent, co
       WAN_PROF(WAN_K_MODEL, s, (patchify_kernel<float><<<grid_for(n), 256, 0, s>>>(
           latent, (float *)patch, B, m.C_in, m.F, m.H, m.W), 0));
     WAN_CHECK_LAUNCH("patchify");
-    WAN_TRY_CUDA(cudaMemsetAsync(X, 0, (size_t)BL * D * sizeof(float), s), "clear token stream");
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = m.C_in * 4; g.A = patch; g.lda = m.C_in * 4;
     g.Bseg[0] = w->patch_w; g.bias[0] = w->patch_b; g.segN = D; g.nseg = 1;
     g.epi = EPI_RESID; g.X = X; g.ldx = D; g.gate = nullptr; g.rows_per_gate = L;
+    g.x_store = 1;
     if ((rc = gemm_any(g, dt, s))) return rc;
   }
   // time embedding (fp32): e = W2 SiLU(W1 sinusoid(t) + b1) + b2; e0 = Wp SiLU(e) + bp

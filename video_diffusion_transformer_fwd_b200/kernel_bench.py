@@ -4,6 +4,7 @@ driver used for ncu captures of one kernel on a small case).
     python -m video_diffusion_transformer_fwd_b200.kernel_bench attention --B 1 --L 16384 --heads 40
     python -m video_diffusion_transformer_fwd_b200.kernel_bench block --config a14b-step --B 2
     python -m video_diffusion_transformer_fwd_b200.kernel_bench block --config a14b-step --F 5 ...
+    python -m video_diffusion_transformer_fwd_b200.kernel_bench model --blocks 0
 
 Prints one JSON line with the mean device time per call (CUDA events on the
 launching stream, after warm-up) and the per-kernel-class times.
@@ -39,7 +40,8 @@ def _time(fn, iters, warmup):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["attention", "block"])
+    ap.add_argument("what", choices=["attention", "block", "model"])
+    ap.add_argument("--blocks", type=int, default=0)
     ap.add_argument("--config", default="a14b-step")
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--L", type=int, default=16384)
@@ -60,6 +62,9 @@ def main():
                           "ms": ms, "tflops": flops / ms / 1e9, "kernels_ms": prof}))
         return
     cfg = configs.get(a.config)
+    if a.what == "model":
+        model(cfg, a)
+        return
     if a.F:
         cfg = dataclasses.replace(cfg, F=a.F)
     cfg = dataclasses.replace(cfg, batch=a.B)
@@ -75,6 +80,41 @@ def main():
                       "tflops": cfg.block_flops() / ms / 1e9,
                       "gemm_tflops": cfg.gemm_flops() / (prof.get("gemm_tc", 0) or float("nan")) / 1e9,
                       "attn_tflops": cfg.self_attn_flops() / (prof.get("attn_self", 0) or float("nan")) / 1e9,
+                      "kernels_ms": prof}))
+
+
+def model(cfg, a):
+    """wan_model_forward on the CFG pair (B = 2) at the config's token grid
+    (latent [16, F, 2H, 2W], text 512 x 4096) with ``--blocks`` blocks; with 0
+    blocks it times the embeddings, head and unpatchify alone."""
+    F = a.F or cfg.F
+    C, text_dim, B = 16, 4096, 2
+    dims = wan.make_model_dims(C, C, F, 2 * cfg.H, 2 * cfg.W, cfg.dim, cfg.heads, cfg.ffn_dim,
+                               cfg.text_len, text_dim, 256, cfg.eps, cfg.dtype)
+    mw = synth.model_weights(C, C, cfg.dim, text_dim, 256, cfg.dtype, "cuda")
+    blocks = wan.make_block_array([synth.block_weights(cfg.dim, cfg.ffn_dim, cfg.dtype, "cuda", i)
+                                   for i in range(a.blocks)]) if a.blocks else wan.make_block_array([])
+    inp = synth.model_inputs(B, C, F, 2 * cfg.H, 2 * cfg.W, cfg.text_len, text_dim, cfg.dtype,
+                             "cuda", same_latent=True)
+    t = torch.full((B,), 900.0, device="cuda")
+    rope = wan.rope_freqs(cfg.head_dim, 1024, cfg.theta)
+    ws = wan.alloc_model_workspace(dims, B)
+    out = torch.empty((B, C, F, 2 * cfg.H, 2 * cfg.W), device="cuda")
+    mwc = wan.make_model_weights(mw)
+    ms, prof = _time(lambda: wan.model_forward(dims, inp["latent"], t, inp["text"], mwc, blocks,
+                                               rope, ws, out=out), a.iters, a.warmup)
+    L = F * cfg.H * cfg.W
+    es = 2 if cfg.dtype == "bf16" else 4
+    D = cfg.dim
+    # bytes the embeddings and head must move at least: latent in, x written once (fp32),
+    # x read by the head LN, its output written and read by the head GEMM, velocity out,
+    # plus every weight once
+    wbytes = sum(v.numel() * v.element_size() for v in mw.values())
+    alg = (B * C * L * 4 * 4 + B * L * D * 4 + B * L * D * 4 + 2 * B * L * D * es
+           + B * C * L * 4 * 4 + inp["text"].numel() * es + wbytes)
+    print(json.dumps({"what": "model", "config": cfg.name, "B": B, "L": L, "blocks": a.blocks,
+                      "ms": ms, "embed_head_algorithmic_bytes": alg,
+                      "embed_head_gbs": alg / ms / 1e6 if a.blocks == 0 else None,
                       "kernels_ms": prof}))
 
 
