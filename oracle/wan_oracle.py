@@ -18,7 +18,9 @@ Sources (the pages that define what is computed):
   loop snippet (classifier-free guidance).
 * [DIGEST] "Wan paper deep dive" (charles2530.github.io), section
   "Video DiT and Flow Matching": token count formula, shared AdaLN MLP with a
-  per-block bias, flow-matching path x_t = t x1 + (1-t) x0 and v = x1 - x0.
+  per-block bias, flow-matching path x_t = t x1 + (1-t) x0 and v = x1 - x0;
+  and its inference-optimisation table (FP8 GEMM: one scale per weight
+  tensor, one per activation token).
 * [TRACE] "Wan2.2 I2V inference trace" (damodev.csdn.net), section 4 "DIT":
   token shapes and the CFG scale meaning (s = 1: prompt only).
 * [DIFFUSERS] "diffusers WanPipeline walkthrough" (huan-yin.github.io),
@@ -35,6 +37,10 @@ Readings taken where the pages are silent:
   the population variance with eps inside the square root.
 * Softmax scale 1/sqrt(head_dim); every Linear has a bias.
 * A query row with zero valid keys (key length 0) outputs zeros.
+* FP8 GEMM: codes are e4m3 ("fn": no infinities, largest finite 448), the
+  scale of a row or tensor is amax / 448, an element's code is the nearest
+  e4m3 value to x * (448 / amax) (ties to even, clamped to +-448), and these
+  decisions are taken in fp32; an all-zero row or tensor gets scale 0.
 
 Every function cites the passage it follows.
 """
@@ -191,6 +197,75 @@ def linear(a: np.ndarray, w: np.ndarray, b) -> np.ndarray:
     return y
 
 
+_linear = linear
+
+
+# --------------------------------------------------------------------------
+# FP8 GEMM ([DIGEST] inference-optimisation table, "FP8 GEMM": per-tensor
+# weight quantization, per-token activation quantization for the GEMMs of the
+# DiT block). Code layout of e4m3 from the OCP 8-bit floating-point format
+# (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 15
+# with mantissa 7 is NaN, there is no infinity).
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each e4m3 byte (NaN for 0x7F and 0xFF)."""
+    c = np.asarray(codes, np.int64) & 0xFF
+    sign = np.where(c >= 128, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(F64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e.astype(F64) - 7))
+    mag = np.where((e == 15) & ((c & 7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest e4m3 value (ties to the even code), magnitudes above 448 clamped
+    to 448. Values are spaced 2^(e-3) within the binade [2^e, 2^(e+1)), e >= -6;
+    below 2^-6 the spacing stays 2^-9 (subnormals)."""
+    x = np.asarray(x, F64)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)
+    step = 2.0 ** (e - 3.0)
+    r = np.round(a / step) * step              # numpy rounds halves to even
+    r = np.minimum(r, E4M3_MAX)
+    return np.copysign(r, x)
+
+
+def quantize_fp8(x, per_row: bool = True):
+    """(codes as values, scales): per row of the last axis (one scale per
+    token) or per tensor. amax, 448 / amax, x * (448 / amax) and amax / 448
+    are each rounded to fp32 as they are formed."""
+    x32 = np.asarray(x, F64).astype(np.float32)
+    if per_row:
+        amax = np.abs(x32).max(axis=-1, keepdims=True) if x32.shape[-1] else np.zeros(x32.shape[:-1] + (1,), np.float32)
+    else:
+        amax = np.array(np.abs(x32).max() if x32.size else 0.0, np.float32)
+    amax = amax.astype(np.float32)
+    nz = amax > 0
+    with np.errstate(divide="ignore"):
+        inv = np.where(nz, np.float32(E4M3_MAX) / np.where(nz, amax, np.float32(1)), np.float32(0)).astype(np.float32)
+    y = (x32 * inv).astype(np.float32)
+    q = e4m3_round(y.astype(F64))
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    return q, scale.astype(F64)
+
+
+def linear_fp8(a, w, b) -> np.ndarray:
+    """FP8 linear layer: a quantized per row, W per tensor, the product of the
+    codes accumulated exactly (fp64), times both scales, plus the bias."""
+    qa, sa = quantize_fp8(a, per_row=True)
+    qw, sw = quantize_fp8(w, per_row=False)
+    y = (qa @ qw.T) * sa * sw
+    if b is not None:
+        y = y + np.asarray(b, F64)
+    return y
+
+
 # --------------------------------------------------------------------------
 # Attention ([WALK] self-attention snippet: global window, no causal mask,
 # key lengths)
@@ -252,9 +327,11 @@ def _mod(w, e0):
     return np.asarray(w["modulation"], F64)[None] + np.asarray(e0, F64)   # [B, 6, D]
 
 
-def self_attn_kv(x, e0, w, heads, grid, eps, theta=1e4):
+def self_attn_kv(x, e0, w, heads, grid, eps, theta=1e4, fp8=False):
     """K (RMSNorm'd, rotated) and V of the self-attention for every row of
-    every sequence: [B, L, n, d] each. Rows interact only through these."""
+    every sequence: [B, L, n, d] each. Rows interact only through these.
+    ``fp8``: the projections are FP8 linear layers."""
+    linear = linear_fp8 if fp8 else _linear
     x = np.asarray(x, F64)
     B, L, D = x.shape
     d = D // heads
@@ -267,7 +344,7 @@ def self_attn_kv(x, e0, w, heads, grid, eps, theta=1e4):
 
 
 def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
-                       theta=1e4, kv=None, intermediates=None):
+                       theta=1e4, kv=None, intermediates=None, fp8=False):
     """Output of one WanAttentionBlock at the token rows ``rows`` of every
     sequence: [B, len(rows), D]. Follows the [WALK] block snippet:
 
@@ -284,7 +361,10 @@ def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
     Self-attention K and V need every row; everything else is row-local, so
     only the requested rows are carried past the key/value projection.
     ``intermediates`` (a dict) receives the per-branch outputs at those rows.
+    ``fp8``: the ten projections (q, k, v, o, cross q, k, v, o, FFN 1 and 2)
+    are FP8 linear layers (``linear_fp8``); everything else is unchanged.
     """
+    linear = linear_fp8 if fp8 else _linear
     x = np.asarray(x, F64)
     ctx = np.asarray(ctx, F64)
     B, L, D = x.shape
@@ -293,7 +373,7 @@ def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
     rows = np.asarray(rows, np.int64)
     m = _mod(w, e0)
     if kv is None:
-        kv = self_attn_kv(x, e0, w, heads, grid, eps, theta)
+        kv = self_attn_kv(x, e0, w, heads, grid, eps, theta, fp8=fp8)
     k_all, v_all = kv
     pos = token_positions(*grid)[rows]
 
@@ -338,11 +418,11 @@ def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
 
 
 def block_forward(x, ctx, ctx_lens, e0, w, heads, grid, eps, theta=1e4,
-                  intermediates=None):
+                  intermediates=None, fp8=False):
     """Full block output [B, L, D] (all rows)."""
     L = np.asarray(x).shape[1]
     return block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps,
-                              np.arange(L), theta=theta, intermediates=intermediates)
+                              np.arange(L), theta=theta, intermediates=intermediates, fp8=fp8)
 
 
 # --------------------------------------------------------------------------
