@@ -24,7 +24,9 @@
  *           self-attention snippet, sampling-loop (CFG) snippet.
  *  [DIGEST] "Wan paper deep dive" (charles2530.github.io), section
  *           "Video DiT and Flow Matching": shared AdaLN MLP with per-block
- *           bias, flow-matching interpolation and velocity.
+ *           bias, flow-matching interpolation and velocity; its
+ *           inference-optimisation table ("FP8 GEMM": per-tensor weight,
+ *           per-token activation quantization).
  */
 #ifndef WAN_H_
 #define WAN_H_
@@ -49,6 +51,7 @@ typedef struct CUstream_st *wan_stream_t;
 /* element types */
 #define WAN_F32  0
 #define WAN_BF16 1
+#define WAN_FP8  2   /* block mode: FP8 GEMMs, bf16 everything else (see wan_dims) */
 
 /* Problem statement of one block call ([WALK]: grid sizes after the (1,2,2)
  * patch embedding, dim, heads, ffn_dim, text length, eps). */
@@ -64,7 +67,13 @@ typedef struct {
                        in float32 with exact fp32 FMA arithmetic.
                        WAN_BF16: matrices, biases, context and intermediates
                        in bfloat16, tensor-core products accumulated in fp32;
-                       norms, softmax, residual stream in fp32.              */
+                       norms, softmax, residual stream in fp32.
+                       WAN_FP8 ([DIGEST] "FP8 GEMM"): as WAN_BF16, except
+                       that the ten projection matrices are e4m3 codes with
+                       one scale each (wan_block_weights.w_scales) and every
+                       projection's input is quantized to e4m3 per token
+                       inside the block; the products run on the FP8 tensor
+                       cores and are accumulated in fp32.                    */
 } wan_dims;
 
 /* Parameters of one WanAttentionBlock ([WALK] block snippet). Pointers marked
@@ -80,6 +89,10 @@ typedef struct {
   const float *cgq, *cgk;                  /* cross-attn q/k RMSNorm gains             */
   const void *w1, *b1;                     /* (dt) FFN in:  [ffn_dim, dim], [ffn_dim]  */
   const void *w2, *b2;                     /* (dt) FFN out: [dim, ffn_dim], [dim]      */
+  const float *w_scales;                   /* WAN_FP8 only (NULL otherwise): [10] scales
+                                              of wq, wk, wv, wo, cwq, cwk, cwv, cwo, w1,
+                                              w2, whose codes (uint8 e4m3) replace the
+                                              matrices above; biases stay bf16          */
 } wan_block_weights;
 
 /* Message describing the last error on the calling thread ("" if none). */
@@ -115,7 +128,10 @@ size_t wan_block_workspace_bytes(const wan_dims *dims, int B);
 #define WAN_WS_MOD   7  /* f32  [B, 6, dim]  modulation + e0                        */
 #define WAN_WS_STATS 8  /* f32  [max(B*L, B*T), 4, dim/256] per-row partial sums of squares of
                            q, k, cross q, cross k (bf16 path) */
-#define WAN_WS_COUNT 9
+#define WAN_WS_A8     9  /* u8 [max(B*L*ffn, B*T*dim)] e4m3 codes of the last quantized GEMM input
+                           (WAN_FP8 only; empty otherwise)                              */
+#define WAN_WS_ASCALE 10 /* f32 [max(B*L, B*T)] their per-row scales (WAN_FP8 only)       */
+#define WAN_WS_COUNT 11
 /* Byte offset of buffer `which` inside the workspace, or (size_t)-1. */
 size_t wan_block_workspace_offset(const wan_dims *dims, int B, int which);
 
@@ -131,8 +147,9 @@ size_t wan_block_workspace_offset(const wan_dims *dims, int B, int which);
  *   keys/values from ctx, first ctx_lens[b] text tokens valid. FFN: Linear,
  *   GELU(tanh), Linear. LayerNorm without affine uses eps inside the sqrt.
  *
- *   dims      problem statement; head_dim must be 128 for WAN_BF16, and one of
- *             32, 64, 128 for WAN_F32. dim % 64 == 0, ffn_dim % 64 == 0.
+ *   dims      problem statement; head_dim must be 128 for WAN_BF16 and
+ *             WAN_FP8, and one of 32, 64, 128 for WAN_F32. dim % 64 == 0,
+ *             ffn_dim % 64 == 0 (WAN_FP8: dim % 256 == 0, ffn_dim % 128 == 0).
  *   B         sequences (2 for a CFG pair: same x, two contexts), >= 1.
  *   x         in/out float32 [B, L, dim], the residual stream.
  *   ctx       (dt) [B, T, dim] projected text tokens.
@@ -198,7 +215,9 @@ typedef struct {
   int text_dim;         /* width of the text encoder features (4096 for umT5)   */
   int freq_dim;         /* sinusoidal time features (256)                        */
   float eps;
-  int dtype;            /* WAN_F32 | WAN_BF16, as in wan_dims                    */
+  int dtype;            /* WAN_F32 | WAN_BF16 | WAN_FP8, as in wan_dims; with
+                           WAN_FP8 the blocks run their FP8 GEMMs and the
+                           embeddings and head are bf16                           */
 } wan_model_dims;
 
 /* (dt) = wan_model_dims.dtype; others float32. */
@@ -234,6 +253,33 @@ int wan_model_forward(const wan_model_dims *dims, int B, const float *latent, co
                       const wan_block_weights *blocks, int num_blocks, const float *rope,
                       int rope_max_pos, float *out, void *workspace, size_t ws_bytes,
                       wan_stream_t stream);
+
+/* wan_quantize_fp8 -- e4m3 quantization ([DIGEST] "FP8 GEMM"), per row (one
+ * scale per token) or per tensor (one scale for all, as for weights).
+ *   src       (src_dtype: WAN_F32 or WAN_BF16) [rows, cols], dense.
+ *   per_row   1: scale[r] for every row; 0: one scale for the whole tensor.
+ *   q         out uint8 [rows, cols] e4m3 codes ("fn" encoding: 1 sign,
+ *             4 exponent bits biased by 7, 3 mantissa bits, largest 448).
+ *   scale     out float32 [rows] (per_row) or [1]: amax / 448.
+ * Rule: code = e4m3(x * (448 / amax)), nearest value with ties to even,
+ * saturating at +-448; 448 / amax, the product and amax / 448 each rounded to
+ * fp32. An all-zero row (or tensor) gets codes 0 and scale 0.
+ * Constraints: cols % 4 == 0 (per row) or rows * cols % 4 == 0 (per tensor).
+ * Errors: WAN_EINVAL (sizes, NULL), WAN_EALIGN, WAN_EUNSUPPORTED. */
+int wan_quantize_fp8(const void *src, int src_dtype, int rows, int cols, int per_row, uint8_t *q,
+                     float *scale, wan_stream_t stream);
+
+/* wan_linear_fp8 -- FP8 linear layer on the tensor cores ([DIGEST] "FP8 GEMM"):
+ *   out[m, n] = (sum_k a[m, k] w[n, k]) * a_scale[m] * w_scale[0] + bias[n]
+ *   a        uint8 e4m3 [M, K], a_scale float32 [M] (per token);
+ *   w        uint8 e4m3 [N, K], w_scale float32 [1] (per tensor), both as
+ *            written by wan_quantize_fp8; bias bf16 [N] or NULL.
+ *   out      float32 [M, N].
+ * Products of codes are exact and accumulated in fp32.
+ * Constraints: K % 128 == 0, N % 32 == 0, M >= 1.
+ * Errors: WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED. */
+int wan_linear_fp8(int M, int N, int K, const uint8_t *a, const float *a_scale, const uint8_t *w,
+                   const float *w_scale, const void *bias, float *out, wan_stream_t stream);
 
 /* wan_attention -- softmax attention, non-causal, every head
  * ([WALK] self-attention snippet: global window, key lengths).
@@ -299,7 +345,8 @@ int wan_selftest_watchdog(wan_stream_t stream);
 #define WAN_K_MISC         8  /* modulation combine, RoPE table               */
 #define WAN_K_ATTN_TC      9  /* tensor-core attention via wan_attention      */
 #define WAN_K_MODEL       10  /* patchify, embeddings, head, unpatchify       */
-#define WAN_K_COUNT       11
+#define WAN_K_QUANT       11  /* e4m3 quantization of GEMM inputs / weights   */
+#define WAN_K_COUNT       12
 int wan_profile_enable(int on);
 int wan_profile_read(int kernel_class, int *launches, double *total_ms);
 

@@ -76,9 +76,12 @@ static int check_dims(const wan_dims *d, int B) {
   if (d->ffn_dim < 64 || d->ffn_dim % 64) return set_error(WAN_EINVAL, "ffn_dim %d must be a positive multiple of 64", d->ffn_dim);
   if (d->text_len < 0) return set_error(WAN_EINVAL, "text_len %d < 0", d->text_len);
   if (!(d->eps >= 0.f)) return set_error(WAN_EINVAL, "eps must be >= 0");
-  if (d->dtype != WAN_F32 && d->dtype != WAN_BF16) return set_error(WAN_EUNSUPPORTED, "dtype %d", d->dtype);
+  if (d->dtype != WAN_F32 && d->dtype != WAN_BF16 && d->dtype != WAN_FP8)
+    return set_error(WAN_EUNSUPPORTED, "dtype %d", d->dtype);
   const int hd = d->dim / d->heads;
-  if (d->dtype == WAN_BF16 && hd != 128) return set_error(WAN_EUNSUPPORTED, "bf16 path needs head_dim 128 (got %d)", hd);
+  if (d->dtype != WAN_F32 && hd != 128) return set_error(WAN_EUNSUPPORTED, "bf16 / fp8 paths need head_dim 128 (got %d)", hd);
+  if (d->dtype == WAN_FP8 && (d->dim % 256 || d->ffn_dim % 128))
+    return set_error(WAN_EUNSUPPORTED, "fp8 path needs dim %% 256 == 0 and ffn_dim %% 128 == 0");
   if (d->dtype == WAN_F32 && hd != 32 && hd != 64 && hd != 128)
     return set_error(WAN_EUNSUPPORTED, "fp32 path needs head_dim 32, 64 or 128 (got %d)", hd);
   const long long L = (long long)d->F * d->H * d->W;
@@ -101,6 +104,8 @@ static WsLayout layout_of(const wan_dims *d, int B) {
       BL * Fh * es,           // H
       (size_t)B * 6 * D * 4,  // MOD
       (BL > (size_t)B * T ? BL : (size_t)B * T) * 4 * (D >= 256 ? D / 256 : 1) * 4,   // STATS: per-row partial sums of squares
+      d->dtype == WAN_FP8 ? (BL * Fh > (size_t)B * T * D ? BL * Fh : (size_t)B * T * D) : 0,   // A8
+      d->dtype == WAN_FP8 ? (BL > (size_t)B * T ? BL : (size_t)B * T) * 4 : 0,                // ASCALE
   };
   size_t o = 0;
   for (int i = 0; i < WAN_WS_COUNT; ++i) {
@@ -109,6 +114,131 @@ static WsLayout layout_of(const wan_dims *d, int B) {
   }
   w.total = o;
   return w;
+}
+
+// ---------------------------------------------------------------- FP8 block
+// The fused bf16 block with every projection on the FP8 tensor cores
+// ("Wan paper deep dive" (charles2530.github.io), inference-optimisation
+// table, "FP8 GEMM"): each projection's input is quantized per token to e4m3
+// (inside the LayerNorm for the three normalised branch inputs, by a row pass
+// for the attention outputs, the FFN hidden and the context), the weights are
+// e4m3 with one scale per matrix, and the GEMM epilogue multiplies by both
+// scales before the bias, q/k-norm, GELU or gated residual.
+static int block_forward_fp8(const wan_dims &d, int B, float *x, const void *ctx, const int *ctx_lens,
+                             const wan_block_weights *w, const float *rope, char *ws, const WsLayout &lay,
+                             const float *mod, cudaStream_t s) {
+  const int L = d.F * d.H * d.W, D = d.dim, T = d.text_len, Fh = d.ffn_dim, hd = D / d.heads, BL = B * L;
+  const size_t es = 2;
+  char *qkv = ws + lay.off[WAN_WS_QKV];
+  void *o = ws + lay.off[WAN_WS_O];
+  void *qc = ws + lay.off[WAN_WS_QC];
+  char *kvc = ws + lay.off[WAN_WS_KVC];
+  void *oc = ws + lay.off[WAN_WS_OC];
+  void *hbuf = ws + lay.off[WAN_WS_H];
+  float *stats = reinterpret_cast<float *>(ws + lay.off[WAN_WS_STATS]);
+  uint8_t *a8 = reinterpret_cast<uint8_t *>(ws + lay.off[WAN_WS_A8]);
+  float *asc = reinterpret_cast<float *>(ws + lay.off[WAN_WS_ASCALE]);
+  const float *wsc = w->w_scales;
+  const int parts = D / 256, sstride = 4 * parts;
+  const float scale = 1.0f / sqrtf((float)hd);
+  int rc;
+  auto gemm8 = [&](GemmArgs &g) -> int {
+    g.fp8 = 1; g.A = a8; g.lda = g.K; g.a_scale = asc;
+    if (!gemm_tc_supported(g)) return set_error(WAN_EUNSUPPORTED, "fp8 GEMM M=%d N=%d K=%d", g.M, g.N, g.K);
+    return WAN_PROF(WAN_K_GEMM_TC, s, gemm_tc(g, s));
+  };
+  auto quant_rows = [&](const void *src, int rows, int cols) -> int {
+    return WAN_PROF(WAN_K_QUANT, s, launch_quant_rows(src, WAN_BF16, (size_t)cols, rows, cols, a8, asc, s));
+  };
+
+  // ---- self-attention
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod_fp8(x, a8, asc, BL, D, L, mod, 0, 1, nullptr, nullptr, d.eps, s)))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = 3 * D; g.K = D;
+    g.Bseg[0] = w->wq; g.Bseg[1] = w->wk; g.Bseg[2] = w->wv;
+    g.bias[0] = w->bq; g.bias[1] = w->bk; g.bias[2] = w->bv;
+    g.b_scale[0] = wsc + 0; g.b_scale[1] = wsc + 1; g.b_scale[2] = wsc + 2;
+    g.segN = D; g.nseg = 3; g.C = qkv; g.ldc = 3 * D; g.epi = EPI_QKNORM;
+    g.gamma[0] = w->gq; g.gamma[1] = w->gk; g.gamma[2] = nullptr;
+    g.ss = stats; g.ss_stride = sstride; g.ss_col[0] = 0; g.ss_col[1] = 1; g.ss_col[2] = -1;
+    g.rope = rope; g.rope_mask = 3; g.F = d.F; g.H = d.H; g.W = d.W; g.head_dim = hd;
+    if ((rc = gemm8(g))) return rc;
+  }
+  if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_scale_rows(qkv + D * es, BL, 3 * D, D, stats + parts, sstride, parts, d.eps, s)))) return rc;
+  {
+    AttnArgs a = {};
+    a.B = B; a.heads = d.heads; a.Lq = L; a.Lk = L; a.d = hd;
+    a.q = qkv; a.ldq = 3 * D; a.k = qkv + D * es; a.ldk = 3 * D; a.v = qkv + 2 * D * es; a.ldv = 3 * D;
+    a.o = o; a.ldo = D; a.scale = scale;
+    a.q_ss = stats; a.q_ss_stride = sstride; a.q_ss_parts = parts; a.q_ss_n = (float)D; a.q_ss_eps = d.eps;
+    if (!attention_tc_supported(a)) return set_error(WAN_EUNSUPPORTED, "fp8 block: self-attention shape");
+    if ((rc = WAN_PROF(WAN_K_ATTN_SELF, s, attention_tc(a, s)))) return rc;
+  }
+  if ((rc = quant_rows(o, BL, D))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = D; g.Bseg[0] = w->wo; g.bias[0] = w->bo; g.b_scale[0] = wsc + 3;
+    g.segN = D; g.nseg = 1;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = mod + 2 * D; g.gate_stride = 6 * D; g.rows_per_gate = L;
+    if ((rc = gemm8(g))) return rc;
+  }
+
+  // ---- cross-attention (ungated)
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod_fp8(x, a8, asc, BL, D, L, nullptr, 0, 0, w->g3, w->b3, d.eps, s)))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = D; g.Bseg[0] = w->cwq; g.bias[0] = w->cbq; g.b_scale[0] = wsc + 4;
+    g.segN = D; g.nseg = 1; g.C = qc; g.ldc = D; g.epi = EPI_QKNORM;
+    g.gamma[0] = w->cgq; g.ss = stats; g.ss_stride = sstride; g.ss_col[0] = 2; g.ss_col[1] = g.ss_col[2] = -1;
+    if ((rc = gemm8(g))) return rc;
+  }
+  if (T > 0) {
+    if ((rc = quant_rows(ctx, B * T, D))) return rc;
+    GemmArgs g = {};
+    g.M = B * T; g.N = 2 * D; g.K = D;
+    g.Bseg[0] = w->cwk; g.Bseg[1] = w->cwv; g.bias[0] = w->cbk; g.bias[1] = w->cbv;
+    g.b_scale[0] = wsc + 5; g.b_scale[1] = wsc + 6;
+    g.segN = D; g.nseg = 2; g.C = kvc; g.ldc = 2 * D; g.epi = EPI_QKNORM;
+    g.gamma[0] = w->cgk; g.gamma[1] = nullptr; g.ss = stats; g.ss_stride = sstride;
+    g.ss_col[0] = 3; g.ss_col[1] = -1; g.ss_col[2] = -1;
+    if ((rc = gemm8(g))) return rc;
+    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_scale_rows(kvc, B * T, 2 * D, D, stats + 3 * parts, sstride, parts, d.eps, s)))) return rc;
+  }
+  {
+    AttnArgs a = {};
+    a.B = B; a.heads = d.heads; a.Lq = L; a.Lk = T; a.d = hd;
+    a.q = qc; a.ldq = D; a.k = kvc; a.ldk = 2 * D; a.v = kvc + D * es; a.ldv = 2 * D;
+    a.o = oc; a.ldo = D; a.k_lens = ctx_lens; a.scale = scale;
+    a.q_ss = stats + 2 * parts; a.q_ss_stride = sstride; a.q_ss_parts = parts; a.q_ss_n = (float)D; a.q_ss_eps = d.eps;
+    if ((rc = run_attention(a, WAN_BF16, s, WAN_K_ATTN_CROSS))) return rc;
+  }
+  if ((rc = quant_rows(oc, BL, D))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = D; g.Bseg[0] = w->cwo; g.bias[0] = w->cbo; g.b_scale[0] = wsc + 7;
+    g.segN = D; g.nseg = 1;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = nullptr; g.rows_per_gate = L;
+    if ((rc = gemm8(g))) return rc;
+  }
+
+  // ---- FFN
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod_fp8(x, a8, asc, BL, D, L, mod, 3, 4, nullptr, nullptr, d.eps, s)))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = Fh; g.K = D; g.Bseg[0] = w->w1; g.bias[0] = w->b1; g.b_scale[0] = wsc + 8;
+    g.segN = Fh; g.nseg = 1; g.epi = EPI_GELU; g.C = hbuf; g.ldc = Fh;
+    if ((rc = gemm8(g))) return rc;
+  }
+  if ((rc = quant_rows(hbuf, BL, Fh))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = Fh; g.Bseg[0] = w->w2; g.bias[0] = w->b2; g.b_scale[0] = wsc + 9;
+    g.segN = D; g.nseg = 1;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = mod + 5 * D; g.gate_stride = 6 * D; g.rows_per_gate = L;
+    if ((rc = gemm8(g))) return rc;
+  }
+  return WAN_OK;
 }
 
 }  // namespace wan
@@ -161,6 +291,10 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
     if (!ptrs[i]) return set_error(WAN_EINVAL, "pointer argument #%zu is NULL", i);
     if (!aligned16(ptrs[i])) return set_error(WAN_EALIGN, "pointer argument #%zu not 16-byte aligned", i);
   }
+  if (dt == WAN_FP8) {
+    if (!w->w_scales) return set_error(WAN_EINVAL, "WAN_FP8 needs w_scales");
+    if (!aligned16(w->w_scales)) return set_error(WAN_EALIGN, "w_scales not 16-byte aligned");
+  }
   if (T > 0 && !ctx) return set_error(WAN_EINVAL, "ctx is NULL");
   if (ctx && !aligned16(ctx)) return set_error(WAN_EALIGN, "ctx not 16-byte aligned");
   if (ctx_lens && !aligned16(ctx_lens)) return set_error(WAN_EALIGN, "ctx_lens not 16-byte aligned");
@@ -182,6 +316,7 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
 
   // m = modulation + e0  (shift, scale, gate, shift2, scale2, gate2)
   if ((rc = WAN_PROF(WAN_K_MISC, s, launch_mod_combine(w->modulation, e0, mod, B, D, s)))) return rc;
+  if (dt == WAN_FP8) return block_forward_fp8(d, B, x, ctx, ctx_lens, w, rope, ws, lay, mod, s);
 
   // ---- self-attention branch: x += m2 * Wo . Attn(RoPE(RMSNorm(q,k)), v)
   // bf16 tensor-core path: the QKV GEMM epilogue accumulates each row's sum of
@@ -289,6 +424,49 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
     if ((rc = run_gemm(g, dt, s))) return rc;
   }
   return WAN_OK;
+}
+
+int wan_quantize_fp8(const void *src, int src_dtype, int rows, int cols, int per_row, uint8_t *q,
+                     float *scale, wan_stream_t stream) {
+  g_msg[0] = 0;
+  if (rows < 0 || cols < 0) return set_error(WAN_EINVAL, "rows %d cols %d", rows, cols);
+  if (src_dtype != WAN_F32 && src_dtype != WAN_BF16) return set_error(WAN_EUNSUPPORTED, "src dtype %d", src_dtype);
+  if (!scale && !(per_row && rows == 0)) return set_error(WAN_EINVAL, "scale is NULL");
+  const size_t n = (size_t)rows * cols;
+  if (n > 0 && (!src || !q)) return set_error(WAN_EINVAL, "NULL tensor");
+  const void *ps[] = {src, q, scale};
+  for (const void *p : ps)
+    if (p && !aligned16(p)) return set_error(WAN_EALIGN, "pointer not 16-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (per_row) {
+    if (cols % 4) return set_error(WAN_EUNSUPPORTED, "per-row quantization needs cols %% 4 == 0");
+    return WAN_PROF(WAN_K_QUANT, s, launch_quant_rows(src, src_dtype, (size_t)cols, rows, cols, q, scale, s));
+  }
+  if (n % 4) return set_error(WAN_EUNSUPPORTED, "per-tensor quantization needs rows * cols %% 4 == 0");
+  return WAN_PROF(WAN_K_QUANT, s, launch_quant_tensor(src, src_dtype, n, q, scale, s));
+}
+
+int wan_linear_fp8(int M, int N, int K, const uint8_t *a, const float *a_scale, const uint8_t *w,
+                   const float *w_scale, const void *bias, float *out, wan_stream_t stream) {
+  g_msg[0] = 0;
+  if (M < 0 || N < 0 || K < 0) return set_error(WAN_EINVAL, "M %d N %d K %d", M, N, K);
+  if (M == 0 || N == 0) return WAN_OK;
+  if (K % 128 || K == 0 || N % 32) return set_error(WAN_EUNSUPPORTED, "fp8 linear needs K %% 128 == 0, N %% 32 == 0");
+  if ((long long)M * N > (long long)INT_MAX * 4) return set_error(WAN_EINVAL, "M * N too large");
+  const void *ps[] = {a, a_scale, w, w_scale, out};
+  for (const void *p : ps) {
+    if (!p) return set_error(WAN_EINVAL, "NULL pointer");
+    if (!aligned16(p)) return set_error(WAN_EALIGN, "pointer not 16-byte aligned");
+  }
+  if (bias && !aligned16(bias)) return set_error(WAN_EALIGN, "bias not 16-byte aligned");
+  GemmArgs g = {};
+  g.M = M; g.N = N; g.K = K; g.A = a; g.lda = K;
+  g.Bseg[0] = w; g.bias[0] = bias; g.segN = N; g.nseg = 1;
+  g.epi = EPI_RESID; g.X = out; g.ldx = N; g.gate = nullptr; g.rows_per_gate = 1; g.x_store = 1;
+  g.fp8 = 1; g.a_scale = a_scale; g.b_scale[0] = w_scale;
+  if (!gemm_tc_supported(g)) return set_error(WAN_EUNSUPPORTED, "fp8 linear M=%d N=%d K=%d", M, N, K);
+  cudaStream_t s = (cudaStream_t)stream;
+  return WAN_PROF(WAN_K_GEMM_TC, s, gemm_tc(g, s));
 }
 
 int wan_attention(int B, int heads, int Lq, int Lk, int head_dim, int dtype, void *q, void *k,

@@ -89,7 +89,7 @@ __device__ __forceinline__ float block_sum(float v, float *red) {
 }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-inline size_t dtype_size(int dt) { return dt == WAN_BF16 ? 2 : 4; }
+inline size_t dtype_size(int dt) { return dt == WAN_F32 ? 4 : 2; }   // WAN_FP8: bf16 intermediates
 
 // ---------------------------------------------------------------- internal kernels API
 
@@ -119,6 +119,9 @@ struct GemmArgs {
   float *X; int ldx;
   const float *gate; int gate_stride; int rows_per_gate;
   int x_store;            // EPI_RESID: x = g * y (overwrite) instead of x += g * y
+  int fp8;                // A and B are e4m3 codes: y = (A B^T) a_scale[m] b_scale[seg] + bias
+  const float *a_scale;   // [M] (device)
+  const float *b_scale[3];  // one device float per weight segment
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
   const float *rope; int rope_mask; int F, H, W; int head_dim;
 };
@@ -156,6 +159,14 @@ int launch_mod_combine(const float *modulation, const float *e0, float *mod, int
 int launch_layernorm_mod(const float *x, void *out, int dtype, int rows, int D, int rows_per_b,
                          const float *mod, int shift_chunk, int scale_chunk,
                          const float *g, const float *beta, float eps, cudaStream_t s);
+// the same with the output quantized per row to e4m3 codes q and scales row_scale
+int launch_layernorm_mod_fp8(const float *x, uint8_t *q, float *row_scale, int rows, int D, int rows_per_b,
+                             const float *mod, int shift_chunk, int scale_chunk,
+                             const float *g, const float *beta, float eps, cudaStream_t s);
+// e4m3 quantization per row (src rows ld elements apart) or per tensor (n elements)
+int launch_quant_rows(const void *src, int dtype, size_t ld, int rows, int cols, uint8_t *q, float *scale,
+                      cudaStream_t s);
+int launch_quant_tensor(const void *src, int dtype, size_t n, uint8_t *q, float *scale, cudaStream_t s);
 // In place on rows of a strided matrix: v = RMSNorm_D(v) * gain, then the 3D
 // RoPE of token (r % L) when rope != NULL.
 int launch_rmsnorm_rope(void *p, int dtype, int rows, int ld, int D, int head_dim,

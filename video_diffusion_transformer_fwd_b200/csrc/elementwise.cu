@@ -8,6 +8,7 @@
 // (charles2530.github.io), "Video DiT and Flow Matching" (Euler in sigma).
 #include "common.cuh"
 
+#include <cuda_fp8.h>
 #include <math.h>
 
 namespace wan {
@@ -33,6 +34,120 @@ int launch_mod_combine(const float *modulation, const float *e0, float *mod, int
 }
 
 // ----------------------------------------------------------------------------
+// e4m3 quantization ("Wan paper deep dive" (charles2530.github.io),
+// inference-optimisation table, "FP8 GEMM"): a row's (or tensor's) scale is
+// amax / 448 and an element's code is the e4m3 value nearest to
+// x * (448 / amax), ties to even, clamped to +-448; both factors and the
+// product are rounded to fp32 as formed. An all-zero row gets scale 0.
+// ----------------------------------------------------------------------------
+constexpr float E4M3_MAX = 448.f;
+
+// four values -> four e4m3 bytes, the first in the lowest byte
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
+
+__device__ __forceinline__ float e4m3_inv_scale(float amax) {
+  return amax > 0.f ? __fdiv_rn(E4M3_MAX, amax) : 0.f;
+}
+
+__device__ __forceinline__ float absmax4(float4 v) {
+  return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+}
+
+__device__ __forceinline__ float block_max(float v, float *red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float t = (lane < nw) ? red[lane] : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t = fmaxf(t, __shfl_xor_sync(0xffffffffu, t, o));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t quant4(float4 v, float inv) {
+  return e4m3x4(__fmul_rn(v.x, inv), __fmul_rn(v.y, inv), __fmul_rn(v.z, inv), __fmul_rn(v.w, inv));
+}
+
+// One CTA per row of src (row stride ld elements): codes [rows, cols], scale [rows].
+template <typename T>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const T *__restrict__ src, size_t ld, int cols,
+                                                         uint8_t *__restrict__ q, float *__restrict__ scale) {
+  __shared__ float red[32];
+  const size_t row = blockIdx.x;
+  const T *sr = src + row * ld;
+  float amax = 0.f;
+  for (int c = threadIdx.x * 4; c < cols; c += 4 * blockDim.x) amax = fmaxf(amax, absmax4(load4(sr + c)));
+  amax = block_max(amax, red);
+  const float inv = e4m3_inv_scale(amax);
+  uint32_t *qr = reinterpret_cast<uint32_t *>(q + row * cols);
+  for (int c = threadIdx.x * 4; c < cols; c += 4 * blockDim.x) qr[c >> 2] = quant4(load4(sr + c), inv);
+  if (threadIdx.x == 0) scale[row] = __fdiv_rn(amax, E4M3_MAX);
+}
+
+// Per-tensor: amax into the scale word (as ordered bits of a non-negative
+// float), then the codes, then the word becomes amax / 448.
+template <typename T>
+__global__ void __launch_bounds__(256) amax_kernel(const T *__restrict__ src, size_t n4, unsigned *amax_bits) {
+  __shared__ float red[32];
+  float amax = 0.f;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x)
+    amax = fmaxf(amax, absmax4(load4(src + 4 * i)));
+  amax = block_max(amax, red);
+  if (threadIdx.x == 0) atomicMax(amax_bits, __float_as_uint(amax));
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) quant_tensor_kernel(const T *__restrict__ src, size_t n4,
+                                                           const unsigned *__restrict__ amax_bits,
+                                                           uint8_t *__restrict__ q) {
+  const float inv = e4m3_inv_scale(__uint_as_float(*amax_bits));
+  uint32_t *q4 = reinterpret_cast<uint32_t *>(q);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x)
+    q4[i] = quant4(load4(src + 4 * i), inv);
+}
+
+__global__ void amax_to_scale_kernel(float *scale) { scale[0] = __fdiv_rn(scale[0], E4M3_MAX); }
+
+int launch_quant_rows(const void *src, int dtype, size_t ld, int rows, int cols, uint8_t *q, float *scale,
+                      cudaStream_t s) {
+  if (cols % 4 || ld % 4) return set_error(WAN_EUNSUPPORTED, "quantize: cols and row stride must be multiples of 4");
+  if (rows == 0 || cols == 0) return WAN_OK;
+  if (dtype == WAN_F32)
+    quant_rows_kernel<float><<<rows, 256, 0, s>>>(static_cast<const float *>(src), ld, cols, q, scale);
+  else
+    quant_rows_kernel<__nv_bfloat16><<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), ld, cols, q, scale);
+  WAN_CHECK_LAUNCH("quant_rows");
+  return WAN_OK;
+}
+
+int launch_quant_tensor(const void *src, int dtype, size_t n, uint8_t *q, float *scale, cudaStream_t s) {
+  if (n % 4) return set_error(WAN_EUNSUPPORTED, "quantize: element count must be a multiple of 4");
+  WAN_TRY_CUDA(cudaMemsetAsync(scale, 0, sizeof(float), s), "quantize: clear amax");
+  if (n == 0) return WAN_OK;
+  const size_t n4 = n / 4;
+  size_t g = (n4 + 255) / 256;
+  if (g > 148 * 8) g = 148 * 8;
+  unsigned *bits = reinterpret_cast<unsigned *>(scale);
+  if (dtype == WAN_F32) {
+    amax_kernel<float><<<(int)g, 256, 0, s>>>(static_cast<const float *>(src), n4, bits);
+    quant_tensor_kernel<float><<<(int)g, 256, 0, s>>>(static_cast<const float *>(src), n4, bits, q);
+  } else {
+    amax_kernel<__nv_bfloat16><<<(int)g, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), n4, bits);
+    quant_tensor_kernel<__nv_bfloat16><<<(int)g, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), n4, bits, q);
+  }
+  amax_to_scale_kernel<<<1, 1, 0, s>>>(scale);
+  WAN_CHECK_LAUNCH("quant_tensor");
+  return WAN_OK;
+}
+
+// ----------------------------------------------------------------------------
 // LayerNorm over D (population variance, eps inside the square root), then
 // either the AdaLN modulation (1 + scale) * u + shift with chunks taken from
 // m[b] (norm1 / norm2), or an affine g * u + beta (norm3). One CTA per row;
@@ -41,11 +156,14 @@ int launch_mod_combine(const float *modulation, const float *e0, float *mod, int
 constexpr int LN_THREADS = 256;
 constexpr int LN_MAXV = 8;          // float4 per thread: D <= 8192
 
+// With OutT = uint8_t the modulated row is quantized to e4m3 with its own
+// scale (written to row_scale), the input of an FP8 GEMM.
 template <typename OutT>
 __global__ void __launch_bounds__(LN_THREADS)
 layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int D, int rows_per_b,
                      const float *__restrict__ mod, int shift_chunk, int scale_chunk,
-                     const float *__restrict__ g, const float *__restrict__ beta, float eps) {
+                     const float *__restrict__ g, const float *__restrict__ beta, float eps,
+                     float *__restrict__ row_scale) {
   __shared__ float red[32];
   const int row = blockIdx.x;
   const float *xr = x + (size_t)row * D;
@@ -79,6 +197,7 @@ layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int D,
     mscale = mod + ((size_t)b * 6 + scale_chunk) * D;
   }
   OutT *orow = out + (size_t)row * D;
+  float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < LN_MAXV; ++i) {
     const int c = threadIdx.x + i * LN_THREADS;
@@ -98,8 +217,24 @@ layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int D,
       u.y = fmaf(u.y, a.y, b.y);
       u.z = fmaf(u.z, a.z, b.z);
       u.w = fmaf(u.w, a.w, b.w);
-      store4(orow + 4 * c, u);
+      if constexpr (sizeof(OutT) == 1) {
+        v[i] = u;
+        amax = fmaxf(amax, absmax4(u));
+      } else {
+        store4(orow + 4 * c, u);
+      }
     }
+  }
+  if constexpr (sizeof(OutT) == 1) {
+    amax = block_max(amax, red);
+    const float inv = e4m3_inv_scale(amax);
+    uint32_t *qr = reinterpret_cast<uint32_t *>(orow);
+#pragma unroll
+    for (int i = 0; i < LN_MAXV; ++i) {
+      const int c = threadIdx.x + i * LN_THREADS;
+      if (c < nv) qr[c] = quant4(v[i], inv);
+    }
+    if (threadIdx.x == 0) row_scale[row] = __fdiv_rn(amax, E4M3_MAX);
   }
 }
 
@@ -110,11 +245,22 @@ int launch_layernorm_mod(const float *x, void *out, int dtype, int rows, int D, 
   if (rows == 0) return WAN_OK;
   if (dtype == WAN_BF16)
     layernorm_mod_kernel<__nv_bfloat16><<<rows, LN_THREADS, 0, s>>>(
-        x, (__nv_bfloat16 *)out, D, rows_per_b, mod, shift_chunk, scale_chunk, g, beta, eps);
+        x, (__nv_bfloat16 *)out, D, rows_per_b, mod, shift_chunk, scale_chunk, g, beta, eps, nullptr);
   else
     layernorm_mod_kernel<float><<<rows, LN_THREADS, 0, s>>>(
-        x, (float *)out, D, rows_per_b, mod, shift_chunk, scale_chunk, g, beta, eps);
+        x, (float *)out, D, rows_per_b, mod, shift_chunk, scale_chunk, g, beta, eps, nullptr);
   WAN_CHECK_LAUNCH("layernorm_mod");
+  return WAN_OK;
+}
+
+int launch_layernorm_mod_fp8(const float *x, uint8_t *q, float *row_scale, int rows, int D, int rows_per_b,
+                             const float *mod, int shift_chunk, int scale_chunk,
+                             const float *g, const float *beta, float eps, cudaStream_t s) {
+  if (D % 4 || D > 4 * LN_MAXV * LN_THREADS) return set_error(WAN_EUNSUPPORTED, "layernorm: D=%d", D);
+  if (rows == 0) return WAN_OK;
+  layernorm_mod_kernel<uint8_t><<<rows, LN_THREADS, 0, s>>>(x, q, D, rows_per_b, mod, shift_chunk, scale_chunk,
+                                                            g, beta, eps, row_scale);
+  WAN_CHECK_LAUNCH("layernorm_mod_fp8");
   return WAN_OK;
 }
 

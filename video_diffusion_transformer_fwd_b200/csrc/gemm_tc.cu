@@ -1,5 +1,10 @@
 // Tensor-core GEMM for sm_100a: C = A B^T (+ bias) with fused epilogues,
-// bf16 operands, fp32 accumulation in TMEM.
+// bf16 operands, fp32 accumulation in TMEM. The FP8 variant takes e4m3
+// operands with one scale per row of A (per token) and one per weight tensor
+// ("Wan paper deep dive" (charles2530.github.io), inference-optimisation
+// table, "FP8 GEMM"): a stage holds 128 e4m3 per row instead of 64 bf16 (the
+// same 128 bytes), and the epilogue multiplies the accumulator by
+// a_scale[m] * b_scale before the bias.
 //
 // Persistent kernel on CTA pairs (clusters of 2, one CTA per SM): each pair
 // computes 256 x 256 output tiles with tcgen05.mma.cta_group::2 (M = 256 split
@@ -40,6 +45,8 @@ constexpr int THREADS = 192;
 constexpr int GROUP_M = 8;               // pair tiles (256 rows) per raster group
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_bf16(2 * BM, BN, 0);
+constexpr uint32_t IDESC8 = idesc_e4m3(2 * BM, BN);
+constexpr int BK8 = 128;                 // e4m3 elements per stage row (128 bytes)
 constexpr int STG_BYTES = 32 * 32 * 4;  // one warp's 32 x 32 fp32 staging tile (128-byte swizzle)
 constexpr int EPI_SMEM = 4 * 2 * STG_BYTES;  // 4 epilogue warps, double-buffered
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_SMEM + 256;
@@ -51,6 +58,7 @@ struct TcParams {
   void *C; int ldc;
   float *X; int ldx;
   const float *gate; int gate_stride; int rows_per_gate; int x_store;
+  const float *a_scale; const float *b_scale[3];      // FP8: per row of A, per weight segment
   // q/k RMSNorm + RoPE epilogue (EPI_QKNORM)
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
   const float *rope; int rope_mask; int L, H, W; int head_dim;
@@ -71,7 +79,7 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t lo16) {
   return __uint_as_float(lo16 << 16);
 }
 
-template <int EPI>
+template <int EPI, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
@@ -150,8 +158,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint32_t fb_local = smem_u32(&full[stage]);
           if (leader) mbar_arrive_expect_tx(fb_local, 2 * STAGE_BYTES);
           const uint32_t fb = mapa_shared(fb_local, 0);
-          tma_load_2d_pair(smem_u32(sA + stage * A_BYTES), &tmA, kb * BK, a_row, fb);
-          tma_load_2d_pair(smem_u32(sB + stage * B_BYTES), bm, kb * BK, b_row, fb);
+          const int kx = kb * (F8 ? BK8 : BK);
+          tma_load_2d_pair(smem_u32(sA + stage * A_BYTES), &tmA, kx, a_row, fb);
+          tma_load_2d_pair(smem_u32(sB + stage * B_BYTES), bm, kx, b_row, fb);
           ++fills[stage];
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -183,9 +192,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           tc_fence_after();
           const uint64_t a0 = desc_kmajor_sw128(smem_u32(sA + stage * A_BYTES));
           const uint64_t b0 = desc_kmajor_sw128(smem_u32(sB + stage * B_BYTES));
+          // 4 MMAs of 32 bytes of K per stage (16 bf16 or 32 e4m3 each):
+          // the descriptor start address advances 32 bytes (2 in 16-byte units)
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            mma_ss_pair(d, a0 + 2 * kk, b0 + 2 * kk, IDESC, (kb | kk) != 0);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            if (F8)
+              mma_ss_pair_f8(d, a0 + 2 * kk, b0 + 2 * kk, IDESC8, (kb | kk) != 0);
+            else
+              mma_ss_pair(d, a0 + 2 * kk, b0 + 2 * kk, IDESC, (kb | kk) != 0);
+          }
           const uint32_t eb = smem_u32(&empty[stage]);
           tc_commit_pair(eb);
           tc_commit_pair(mapa_shared(eb, 1));
@@ -218,6 +233,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int seg = n0 / p.segN;
       const __nv_bfloat16 *bias = static_cast<const __nv_bfloat16 *>(p.bias[seg]);
       const int nn0 = n0 - seg * p.segN;
+      float rs = 1.f;                        // FP8: dequantization factor of this row
+      if (F8) rs = (m < p.M ? p.a_scale[m] : 0.f) * *p.b_scale[seg];
       // q/k RMSNorm + RoPE epilogue: per-row sum of squares of y, gamma, rotation
       float sq = 0.f;
       int ss_col = -1, tpos = 0, hpos = 0, wpos = 0;
@@ -256,8 +273,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const uint32_t w[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            v[j4 * 8 + 2 * e] = __uint_as_float(r[j4 * 8 + 2 * e]) + bf16_bits_to_float(w[e] & 0xFFFFu);
-            v[j4 * 8 + 2 * e + 1] = __uint_as_float(r[j4 * 8 + 2 * e + 1]) + bf16_bits_to_float(w[e] >> 16);
+            if (F8) {
+              v[j4 * 8 + 2 * e] = fmaf(__uint_as_float(r[j4 * 8 + 2 * e]), rs, bf16_bits_to_float(w[e] & 0xFFFFu));
+              v[j4 * 8 + 2 * e + 1] = fmaf(__uint_as_float(r[j4 * 8 + 2 * e + 1]), rs, bf16_bits_to_float(w[e] >> 16));
+            } else {
+              v[j4 * 8 + 2 * e] = __uint_as_float(r[j4 * 8 + 2 * e]) + bf16_bits_to_float(w[e] & 0xFFFFu);
+              v[j4 * 8 + 2 * e + 1] = __uint_as_float(r[j4 * 8 + 2 * e + 1]) + bf16_bits_to_float(w[e] >> 16);
+            }
           }
         }
         if (EPI == EPI_RESID) {
@@ -351,12 +373,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
-template <int EPI>
+template <int EPI, bool F8>
 int launch(const CUtensorMap &ta, const CUtensorMap *tb, const CUtensorMap &tx, const TcParams &p,
            cudaStream_t s) {
   static int max_pairs = 0;         // per process; the attribute is per function
   if (!max_pairs) {
-    WAN_TRY_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
+    WAN_TRY_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
                  "gemm_tc smem attribute");
     cudaLaunchConfig_t qc = {};
     cudaLaunchAttribute qa[1];
@@ -368,7 +390,7 @@ int launch(const CUtensorMap &ta, const CUtensorMap *tb, const CUtensorMap &tx, 
     qc.attrs = qa;
     qc.numAttrs = 1;
     int clusters = 0;
-    WAN_TRY_CUDA(cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<EPI>, &qc), "gemm_tc occupancy");
+    WAN_TRY_CUDA(cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<EPI, F8>, &qc), "gemm_tc occupancy");
     max_pairs = clusters > 0 ? clusters : sm_count() / 2;
   }
   const int pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
@@ -382,14 +404,20 @@ int launch(const CUtensorMap &ta, const CUtensorMap *tb, const CUtensorMap &tx, 
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  WAN_TRY_CUDA(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI>, ta, tb[0], tb[1], tb[2], tx, p), "gemm_tc launch");
+  WAN_TRY_CUDA(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI, F8>, ta, tb[0], tb[1], tb[2], tx, p), "gemm_tc launch");
   return WAN_OK;
 }
 }  // namespace
 
 bool gemm_tc_supported(const GemmArgs &g) {
   if (g.epi == EPI_SILU) return false;
-  if (g.M < 1 || g.N < 32 || g.K < BK || g.K % BK || g.N % 32) return false;
+  const int bk = g.fp8 ? BK8 : BK;
+  if (g.M < 1 || g.N < 32 || g.K < bk || g.K % bk || g.N % 32) return false;
+  if (g.fp8) {
+    if (!g.a_scale || g.lda % 16) return false;
+    for (int i = 0; i < g.nseg; ++i)
+      if (!g.b_scale[i]) return false;
+  }
   if (g.nseg < 1 || g.nseg > 3 || g.segN * g.nseg != g.N) return false;
   if (g.nseg > 1 && g.segN % BN) return false;
   if (g.lda % 8) return false;
@@ -411,18 +439,23 @@ bool gemm_tc_supported(const GemmArgs &g) {
 int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   if (!gemm_tc_supported(g)) return set_error(WAN_EUNSUPPORTED, "gemm_tc: M=%d N=%d K=%d", g.M, g.N, g.K);
   CUtensorMap ta, tb[3];
-  int rc = encode_tmap_2d_bf16(&ta, g.A, g.K, g.M, (uint64_t)g.lda * 2, BK, BM);
+  int rc = g.fp8 ? encode_tmap_2d_u8(&ta, g.A, g.K, g.M, (uint64_t)g.lda, BK8, BM)
+                 : encode_tmap_2d_bf16(&ta, g.A, g.K, g.M, (uint64_t)g.lda * 2, BK, BM);
   if (rc) return rc;
   for (int i = 0; i < 3; ++i) {
     const int si = i < g.nseg ? i : 0;
-    if ((rc = encode_tmap_2d_bf16(&tb[i], g.Bseg[si], g.K, g.segN, (uint64_t)g.K * 2, BK, BN / 2))) return rc;
+    rc = g.fp8 ? encode_tmap_2d_u8(&tb[i], g.Bseg[si], g.K, g.segN, (uint64_t)g.K, BK8, BN / 2)
+               : encode_tmap_2d_bf16(&tb[i], g.Bseg[si], g.K, g.segN, (uint64_t)g.K * 2, BK, BN / 2);
+    if (rc) return rc;
   }
   TcParams p = {};
   p.M = g.M; p.N = g.N; p.K = g.K; p.segN = g.segN;
   p.num_m = (g.M + 2 * BM - 1) / (2 * BM);
   p.num_n = (g.N + BN - 1) / BN;
   p.num_tiles = p.num_m * p.num_n;
-  p.num_k = g.K / BK;
+  p.num_k = g.K / (g.fp8 ? BK8 : BK);
+  p.a_scale = g.a_scale;
+  for (int i = 0; i < 3; ++i) p.b_scale[i] = g.fp8 ? g.b_scale[i < g.nseg ? i : 0] : nullptr;
   for (int i = 0; i < 3; ++i) p.bias[i] = i < g.nseg ? g.bias[i] : nullptr;
   p.C = g.C; p.ldc = g.ldc; p.X = g.X; p.ldx = g.ldx;
   p.gate = g.gate; p.gate_stride = g.gate_stride; p.rows_per_gate = g.rows_per_gate > 0 ? g.rows_per_gate : 1;
@@ -438,11 +471,19 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   p.watchdog = watchdog_ptr();
   CUtensorMap tx = ta;
   if (g.epi == EPI_RESID && (rc = encode_tmap_2d_f32(&tx, g.X, g.N, g.M, (uint64_t)g.ldx * 4, 32, 32))) return rc;
+  if (g.fp8) {
+    switch (g.epi) {
+      case EPI_STORE: return launch<EPI_STORE, true>(ta, tb, tx, p, s);
+      case EPI_GELU: return launch<EPI_GELU, true>(ta, tb, tx, p, s);
+      case EPI_QKNORM: return launch<EPI_QKNORM, true>(ta, tb, tx, p, s);
+      default: return launch<EPI_RESID, true>(ta, tb, tx, p, s);
+    }
+  }
   switch (g.epi) {
-    case EPI_STORE: return launch<EPI_STORE>(ta, tb, tx, p, s);
-    case EPI_GELU: return launch<EPI_GELU>(ta, tb, tx, p, s);
-    case EPI_QKNORM: return launch<EPI_QKNORM>(ta, tb, tx, p, s);
-    default: return launch<EPI_RESID>(ta, tb, tx, p, s);
+    case EPI_STORE: return launch<EPI_STORE, false>(ta, tb, tx, p, s);
+    case EPI_GELU: return launch<EPI_GELU, false>(ta, tb, tx, p, s);
+    case EPI_QKNORM: return launch<EPI_QKNORM, false>(ta, tb, tx, p, s);
+    default: return launch<EPI_RESID, false>(ta, tb, tx, p, s);
   }
 }
 

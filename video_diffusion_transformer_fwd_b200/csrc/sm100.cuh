@@ -221,6 +221,20 @@ __device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t adesc, uin
         "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z) : "memory");
 }
 
+// The same pair MMA on 8-bit operands (kind::f8f6f4; formats in the
+// instruction descriptor), fp32 accumulate. One instruction consumes K = 32
+// bytes of each operand row, like K = 16 of kind::f16.
+__device__ __forceinline__ void mma_ss_pair_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  const uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, {%5, %6, %7, %8, %9, %10, %11, %12}, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate),
+        "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z) : "memory");
+}
+
 // K-major operand in 128-byte-swizzled rows (TMA SWIZZLE_128B, 64 bf16 per
 // row, 8-row groups 1024 bytes apart). Tile base must be 1024-byte aligned.
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
@@ -248,6 +262,12 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t 
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn_major << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// kind::f8f6f4 instruction descriptor: e4m3 x e4m3 -> f32 (A and B format
+// fields 0 = E4M3), M x N, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread t gets lane (base + t).
@@ -297,6 +317,8 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // Host side: cuTensorMapEncodeTiled fetched through the runtime (no libcuda link).
 int encode_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                         uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
+int encode_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
 int encode_tmap_2d_f32(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
 int encode_tmap_3d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,

@@ -43,6 +43,11 @@ int encode_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint
   return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, inner, rows, row_stride_bytes, box_inner, box_rows);
 }
 
+int encode_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                      uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows) {
+  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, rows, row_stride_bytes, box_inner, box_rows);
+}
+
 int encode_tmap_2d_f32(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows) {
   return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, inner, rows, row_stride_bytes, box_inner, box_rows);

@@ -15,15 +15,15 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libwan.so")
 
 WAN_OK, WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED, WAN_ECUDA, WAN_ETIMEOUT = 0, -1, -2, -3, -4, -5
-WAN_F32, WAN_BF16 = 0, 1
+WAN_F32, WAN_BF16, WAN_FP8 = 0, 1, 2
 WAN_NOALLOC_WORKSPACE_BYTES = 16 << 20
 (WAN_WS_ACT, WAN_WS_QKV, WAN_WS_O, WAN_WS_QC, WAN_WS_KVC, WAN_WS_OC, WAN_WS_H, WAN_WS_MOD,
- WAN_WS_STATS) = range(9)
+ WAN_WS_STATS, WAN_WS_A8, WAN_WS_ASCALE) = range(11)
 (WAN_K_GEMM_TC, WAN_K_GEMM_SIMT, WAN_K_ATTN_SELF, WAN_K_ATTN_CROSS, WAN_K_ATTN_SIMT, WAN_K_LAYERNORM,
- WAN_K_QKNORM_ROPE, WAN_K_EULER, WAN_K_MISC, WAN_K_ATTN_TC, WAN_K_MODEL) = range(11)
-WAN_K_COUNT = 11
+ WAN_K_QKNORM_ROPE, WAN_K_EULER, WAN_K_MISC, WAN_K_ATTN_TC, WAN_K_MODEL, WAN_K_QUANT) = range(12)
+WAN_K_COUNT = 12
 KERNEL_CLASS_NAMES = ("gemm_tc", "gemm_simt", "attn_self", "attn_cross", "attn_simt", "layernorm",
-                      "qknorm_rope", "euler_cfg", "misc", "attn_tc", "model")
+                      "qknorm_rope", "euler_cfg", "misc", "attn_tc", "model", "quant")
 STATUS_NAMES = {0: "WAN_OK", -1: "WAN_EINVAL", -2: "WAN_EALIGN", -3: "WAN_EUNSUPPORTED",
                 -4: "WAN_ECUDA", -5: "WAN_ETIMEOUT"}
 
@@ -42,7 +42,9 @@ class wan_dims(ctypes.Structure):
 
 WEIGHT_FIELDS = ("modulation", "wq", "bq", "wk", "bk", "wv", "bv", "wo", "bo", "gq", "gk",
                  "g3", "b3", "cwq", "cbq", "cwk", "cbk", "cwv", "cbv", "cwo", "cbo",
-                 "cgq", "cgk", "w1", "b1", "w2", "b2")
+                 "cgq", "cgk", "w1", "b1", "w2", "b2", "w_scales")
+# the ten projection matrices, in the order of wan_block_weights.w_scales
+FP8_MATRICES = ("wq", "wk", "wv", "wo", "cwq", "cwk", "cwv", "cwo", "w1", "w2")
 
 
 class wan_block_weights(ctypes.Structure):
@@ -86,6 +88,8 @@ _SIGS = {
     "wan_selftest_watchdog": (_c_int, [_vp]),
     "wan_profile_read": (_c_int, [_c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]),
     "wan_model_workspace_bytes": (_sz, [ctypes.POINTER(wan_model_dims), _c_int]),
+    "wan_quantize_fp8": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
+    "wan_linear_fp8": (_c_int, [_c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "wan_model_forward": (_c_int, [ctypes.POINTER(wan_model_dims), _c_int, _vp, _vp, _vp, _vp,
                                    ctypes.POINTER(wan_model_weights),
                                    ctypes.POINTER(wan_block_weights), _c_int, _vp, _c_int, _vp,
@@ -173,6 +177,14 @@ def wan_model_forward(dims, B, latent, t, text, ctx_lens, weights, blocks, num_b
                                     out, workspace, ws_bytes, stream)
 
 
+def wan_quantize_fp8(src, src_dtype, rows, cols, per_row, q, scale, stream):
+    return load().wan_quantize_fp8(src, src_dtype, rows, cols, per_row, q, scale, stream)
+
+
+def wan_linear_fp8(M, N, K, a, a_scale, w, w_scale, bias, out, stream):
+    return load().wan_linear_fp8(M, N, K, a, a_scale, w, w_scale, bias, out, stream)
+
+
 def wan_device_status(stream):
     return load().wan_device_status(stream)
 
@@ -226,8 +238,11 @@ def dtype_code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+DTYPE_CODES = {"bf16": WAN_BF16, "f32": WAN_F32, "fp8": WAN_FP8}
+
+
 def make_dims(F, H, W, dim, heads, ffn_dim, text_len, eps=1e-6, dtype="bf16") -> wan_dims:
-    code = {"bf16": WAN_BF16, "f32": WAN_F32}[dtype] if isinstance(dtype, str) else int(dtype)
+    code = DTYPE_CODES[dtype] if isinstance(dtype, str) else int(dtype)
     return wan_dims(F, H, W, dim, heads, ffn_dim, text_len, eps, code)
 
 
@@ -238,9 +253,48 @@ def dims_of(cfg) -> wan_dims:
 
 def make_weights(w: dict) -> wan_block_weights:
     for n in WEIGHT_FIELDS:
-        if not w[n].is_contiguous():
+        if w.get(n) is not None and not w[n].is_contiguous():
             raise ValueError(f"weight {n} must be contiguous")
-    return wan_block_weights(*[w[n].data_ptr() for n in WEIGHT_FIELDS])
+    return wan_block_weights(*[_ptr(w.get(n)) for n in WEIGHT_FIELDS])
+
+
+def quantize_fp8(t, per_row=True, stream=None):
+    """e4m3 codes (uint8, same shape) and float32 scales ([rows] or [1]) of a
+    float32 / bf16 tensor; rows are the last axis."""
+    torch = _torch()
+    cols = t.shape[-1] if t.dim() else 1
+    rows = t.numel() // cols if cols else 0
+    q = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
+    sc = torch.empty((rows if per_row else 1,), dtype=torch.float32, device=t.device)
+    check(wan_quantize_fp8(t.data_ptr(), dtype_code(t), rows, cols, 1 if per_row else 0,
+                           q.data_ptr(), sc.data_ptr(), _stream(stream)))
+    return q, sc
+
+
+def linear_fp8(a, a_scale, w, w_scale, bias=None, out=None, stream=None):
+    """out = (a w^T) a_scale[m] w_scale + bias, float32 [M, N]."""
+    torch = _torch()
+    M, K = a.shape
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=a.device)
+    check(wan_linear_fp8(M, N, K, a.data_ptr(), a_scale.data_ptr(), w.data_ptr(), w_scale.data_ptr(),
+                         _ptr(bias), out.data_ptr(), _stream(stream)))
+    return out
+
+
+def quantize_block_weights(w: dict, stream=None) -> dict:
+    """An FP8 copy of a bf16 block weight dict: the ten projection matrices
+    become e4m3 codes and ``w_scales`` holds their ten per-tensor scales."""
+    torch = _torch()
+    out = dict(w)
+    scales = torch.empty(10, dtype=torch.float32, device=w["wq"].device)
+    for i, n in enumerate(FP8_MATRICES):
+        q, sc = quantize_fp8(w[n], per_row=False, stream=stream)
+        out[n] = q
+        scales[i:i + 1].copy_(sc)
+    out["w_scales"] = scales
+    return out
 
 
 def rope_freqs(head_dim, max_pos=1024, theta=1e4, device="cuda", stream=None):
@@ -313,7 +367,7 @@ def device_status(stream=None) -> int:
 
 def make_model_dims(C_in, C_out, F, H, W, dim, heads, ffn_dim, text_len, text_dim, freq_dim=256,
                     eps=1e-6, dtype="bf16") -> wan_model_dims:
-    code = {"bf16": WAN_BF16, "f32": WAN_F32}[dtype] if isinstance(dtype, str) else int(dtype)
+    code = DTYPE_CODES[dtype] if isinstance(dtype, str) else int(dtype)
     return wan_model_dims(C_in, C_out, F, H, W, dim, heads, ffn_dim, text_len, text_dim, freq_dim,
                           eps, code)
 
