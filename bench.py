@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--config", default="a14b-step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 GEMM mode of the blocks (e4m3 projections, bf16 attention); not the default")
     return ap.parse_args()
 
 
@@ -134,11 +136,11 @@ class OracleSample:
     fixed per-call cost of the text K/V projection). Inputs are drawn once
     by the seeded generators; only the oracle calls are timed."""
 
-    def __init__(self, cfg, seed=0, r_kv=512, r_q=2):
+    def __init__(self, cfg, seed=0, r_kv=512, r_q=2, fp8=False):
         import numpy as np
 
         from video_diffusion_transformer_fwd_b200 import synth
-        self.cfg, self.r_kv, self.r_q = cfg, r_kv, r_q
+        self.cfg, self.r_kv, self.r_q, self.fp8 = cfg, r_kv, r_q, fp8
         w = synth.block_weights(cfg.dim, cfg.ffn_dim, cfg.dtype, "cpu", seed)
         self.w64 = {k: synth.to_numpy64(v) for k, v in w.items()}
         acts = synth.block_activations(1, r_kv, cfg.dim, cfg.text_len, cfg.dtype, "cpu", seed + 100)
@@ -155,7 +157,8 @@ class OracleSample:
         from oracle import wan_oracle as O
         cfg, r_kv, r_q = self.cfg, self.r_kv, self.r_q
         t0 = time.perf_counter()
-        k, v = O.self_attn_kv(self.x, self.e0, self.w64, cfg.heads, (1, 1, r_kv), cfg.eps, cfg.theta)
+        k, v = O.self_attn_kv(self.x, self.e0, self.w64, cfg.heads, (1, 1, r_kv), cfg.eps, cfg.theta,
+                              fp8=self.fp8)
         t_kv = time.perf_counter() - t0
         # full-length keys/values (rows repeated: the attention cost depends only on L)
         kf = np.tile(k, (1, self.reps, 1, 1))[:, :cfg.L]
@@ -165,12 +168,12 @@ class OracleSample:
         for r in (r_q, 2 * r_q):
             t0 = time.perf_counter()
             O.block_forward_rows(self.xq, self.ctx, None, self.e0, self.w64, cfg.heads, grid, cfg.eps,
-                                 np.arange(r), theta=cfg.theta, kv=(kf, vf))
+                                 np.arange(r), theta=cfg.theta, kv=(kf, vf), fp8=self.fp8)
             times.append(time.perf_counter() - t0)
         per_row = max((times[1] - times[0]) / r_q, 0.0)
         fixed = max(times[0] - per_row * r_q, 0.0)
         est = t_kv * cfg.L / r_kv + fixed + per_row * cfg.L
-        detail = (f"fp64 oracle on one block forward of the workload's block shape (one sequence): "
+        detail = (("FP8-GEMM " if self.fp8 else "") + f"fp64 oracle on one block forward of the workload's block shape (one sequence): "
                   f"LN + K/V projection timed on {r_kv} rows (scaled x{cfg.L / r_kv:.1f}); the rest "
                   f"of the block timed for {r_q} and {2 * r_q} query rows attending over all {cfg.L} "
                   f"keys (per-row cost x{cfg.L}, plus the per-call text K/V projection); "
@@ -264,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
     cfg = configs.get(args.config)
-    st = DenoiseStep(cfg, seed=1000 * rank, device=dev)
+    st = DenoiseStep(cfg, seed=1000 * rank, device=dev, fp8=args.fp8)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -359,18 +362,23 @@ def run_ours(args, rank, world, local_rank):
                     "traffic": traffic, "avg_launch_ms": avg_ms,
                     "algorithmic_flops_per_launch": attn_flops_launch}
     elif dom == "gemm_tc" and gemm_n:
+        gpk = peak_sust * (2.0 if args.fp8 else 1.0)
         roofline = {"kernel": "gemm_tc (all block GEMMs)", "bound": "tensor", "achieved": gemm_tflops,
-                    "peak": peak_sust, "unit": "TFLOP/s", "frac": gemm_tflops / peak_sust,
-                    "peak_source": f"{peak_src} bf16 sustained", "traffic": None}
+                    "peak": gpk, "unit": "TFLOP/s", "frac": gemm_tflops / gpk,
+                    "peak_source": f"{peak_src} bf16 sustained" + (" x 2 (fp8 / bf16 nominal ratio)" if args.fp8 else ""),
+                    "traffic": None}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8 e4m3 GEMMs (per-token / per-tensor scales), bf16 attention" if args.fp8 else "bf16",
+        "data": "synthetic",
         "impl": "ours",
         "config": workload_config(cfg, world),
         "attention_tflops": attn_tflops, "gemm_tflops": gemm_tflops,
         "attention_frac_of_2250": None if attn_tflops is None else attn_tflops / 2250.0,
         "gemm_frac_of_2250": None if gemm_tflops is None else gemm_tflops / 2250.0,
+        "gemm_frac_of_fp8_4500": None if (gemm_tflops is None or not args.fp8) else gemm_tflops / 4500.0,
         "kernel_ms_per_step": {k: v[1] / args.steps for k, v in prof.items() if v[0]},
         "gpu_launches": sum(v[0] for v in prof.values()),
         "roofline": roofline,
@@ -379,7 +387,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
     }
     if world == 1 and not args.no_cpu_baseline:
-        ms, detail = OracleSample(cfg, seed=0).run()
+        ms, detail = OracleSample(cfg, seed=0, fp8=args.fp8).run()
         line["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": cpu_cores(),
                                 "blas_threads": blas_threads(), "kind": "oracle", "sample": detail}
     print(json.dumps(line), flush=True)

@@ -45,7 +45,7 @@ def _codes_equal(q_gpu, q_ref):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("rows,cols", [(1, 4), (37, 300), (5, 13824), (300, 5120)])
+@pytest.mark.parametrize("rows,cols", [(1, 4), (37, 300), (64, 1024), (5, 13824), (300, 5120)])
 def test_quantize_rows_bit_exact(dtype, rows, cols):
     x = _rows_input(rows, cols, dtype, rows * 7 + cols)
     q, sc = wan.quantize_fp8(x, per_row=True)

@@ -91,6 +91,49 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const T *__restrict__ s
   if (threadIdx.x == 0) scale[row] = __fdiv_rn(amax, E4M3_MAX);
 }
 
+// The same with the row held in registers (one read of the row from DRAM):
+// bf16 rows of up to 8 * CH * 256 elements, cols % 8 == 0, 16-byte loads.
+template <int CH>
+__global__ void __launch_bounds__(256) quant_rows_reg_kernel(const __nv_bfloat16 *__restrict__ src, size_t ld,
+                                                             int cols, uint8_t *__restrict__ q,
+                                                             float *__restrict__ scale) {
+  __shared__ float red[32];
+  const size_t row = blockIdx.x;
+  const __nv_bfloat16 *sr = src + row * ld;
+  uint4 raw[CH];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < CH; ++i) {
+    const int c = (threadIdx.x + i * 256) * 8;
+    raw[i] = c < cols ? *reinterpret_cast<const uint4 *>(sr + c) : make_uint4(0, 0, 0, 0);
+    const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[e] << 16)), fabsf(__uint_as_float(w4[e] & 0xFFFF0000u))));
+  }
+  amax = block_max(amax, red);
+  const float inv = e4m3_inv_scale(amax);
+  uint8_t *qr = q + row * cols;
+#pragma unroll
+  for (int i = 0; i < CH; ++i) {
+    const int c = (threadIdx.x + i * 256) * 8;
+    if (c < cols) {
+      const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+      float f[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        f[2 * e] = __uint_as_float(w4[e] << 16);
+        f[2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+      }
+      uint2 o;
+      o.x = quant4(make_float4(f[0], f[1], f[2], f[3]), inv);
+      o.y = quant4(make_float4(f[4], f[5], f[6], f[7]), inv);
+      *reinterpret_cast<uint2 *>(qr + c) = o;
+    }
+  }
+  if (threadIdx.x == 0) scale[row] = __fdiv_rn(amax, E4M3_MAX);
+}
+
 // Per-tensor: amax into the scale word (as ordered bits of a non-negative
 // float), then the codes, then the word becomes amax / 448.
 template <typename T>
@@ -119,7 +162,17 @@ int launch_quant_rows(const void *src, int dtype, size_t ld, int rows, int cols,
                       cudaStream_t s) {
   if (cols % 4 || ld % 4) return set_error(WAN_EUNSUPPORTED, "quantize: cols and row stride must be multiples of 4");
   if (rows == 0 || cols == 0) return WAN_OK;
-  if (dtype == WAN_F32)
+  const bool reg = dtype == WAN_BF16 && cols % 8 == 0 && ld % 8 == 0 &&
+                   (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && cols <= 8 * 8 * 256;
+  if (reg) {
+    const int ch = (cols + 2047) / 2048;         // 16-byte chunks per thread
+    if (ch <= 1)
+      quant_rows_reg_kernel<1><<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), ld, cols, q, scale);
+    else if (ch <= 3)
+      quant_rows_reg_kernel<3><<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), ld, cols, q, scale);
+    else
+      quant_rows_reg_kernel<8><<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), ld, cols, q, scale);
+  } else if (dtype == WAN_F32)
     quant_rows_kernel<float><<<rows, 256, 0, s>>>(static_cast<const float *>(src), ld, cols, q, scale);
   else
     quant_rows_kernel<__nv_bfloat16><<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), ld, cols, q, scale);

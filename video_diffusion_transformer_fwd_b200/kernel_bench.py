@@ -42,6 +42,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("what", choices=["attention", "block", "model"])
     ap.add_argument("--blocks", type=int, default=0)
+    ap.add_argument("--fp8", action="store_true", help="block: FP8 GEMM mode")
     ap.add_argument("--config", default="a14b-step")
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--L", type=int, default=16384)
@@ -70,13 +71,16 @@ def main():
     cfg = dataclasses.replace(cfg, batch=a.B)
     dims = wan.dims_of(cfg)
     w = synth.block_weights(cfg.dim, cfg.ffn_dim, cfg.dtype, "cuda", 0)
+    if a.fp8:
+        dims.dtype = wan.WAN_FP8
+        w = wan.quantize_block_weights(w)
     acts = synth.block_activations(a.B, cfg.L, cfg.dim, cfg.text_len, cfg.dtype, "cuda", 100)
     rope = wan.rope_freqs(cfg.head_dim, 1024, cfg.theta)
     ws = wan.alloc_workspace(dims, a.B)
     cw = wan.make_weights(w)
     ms, prof = _time(lambda: wan.block_forward(dims, acts["x"], acts["ctx"], acts["e0"], cw, rope, ws),
                      a.iters, a.warmup)
-    print(json.dumps({"what": "block", "config": cfg.name, "B": a.B, "L": cfg.L, "ms": ms,
+    print(json.dumps({"what": "block", "config": cfg.name, "B": a.B, "L": cfg.L, "fp8": a.fp8, "ms": ms,
                       "tflops": cfg.block_flops() / ms / 1e9,
                       "gemm_tflops": cfg.gemm_flops() / (prof.get("gemm_tc", 0) or float("nan")) / 1e9,
                       "attn_tflops": cfg.self_attn_flops() / (prof.get("attn_self", 0) or float("nan")) / 1e9,
