@@ -298,6 +298,68 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
 
 
 # --------------------------------------------------------------------------
+# 8-bit attention ([DIGEST] inference-optimisation table, "8-bit
+# FlashAttention": int8 for S = Q K^T, FP8 for O = P V, fp32 accumulation
+# across key blocks). Readings where the page is silent: q is quantized per
+# token and head (scale amax/127 over the head's d values), k per head over
+# all keys of the sequence, v to e4m3 per head and channel over all keys
+# (the channel scale factors out of P V), and P = exp(s - max) in (0, 1] is
+# rounded to e4m3; the row normaliser is the exact sum of P. int8 codes are
+# round-half-even of x * (127 / amax), clamped to +-127, decided in fp32.
+# --------------------------------------------------------------------------
+
+I8_MAX = 127.0
+
+
+def quantize_int8(x, axes):
+    """(codes as values, scales) with one scale per slice over ``axes``
+    (kept as size-1 axes): amax, 127 / amax, x * (127 / amax) and amax / 127
+    each rounded to fp32 as formed; an all-zero slice gets codes 0, scale 0."""
+    x32 = np.asarray(x, F64).astype(np.float32)
+    amax = np.abs(x32).max(axis=axes, keepdims=True).astype(np.float32)
+    nz = amax > 0
+    inv = np.where(nz, np.float32(I8_MAX) / np.where(nz, amax, np.float32(1)), np.float32(0)).astype(np.float32)
+    y = (x32 * inv).astype(np.float32).astype(F64)
+    q = np.clip(np.rint(y), -I8_MAX, I8_MAX)
+    return q, (amax / np.float32(I8_MAX)).astype(np.float32).astype(F64)
+
+
+def quantize_fp8_axes(x, axes):
+    """e4m3 codes with one scale per slice over ``axes`` (the rule of
+    ``quantize_fp8``)."""
+    x32 = np.asarray(x, F64).astype(np.float32)
+    amax = np.abs(x32).max(axis=axes, keepdims=True).astype(np.float32)
+    nz = amax > 0
+    inv = np.where(nz, np.float32(E4M3_MAX) / np.where(nz, amax, np.float32(1)), np.float32(0)).astype(np.float32)
+    y = (x32 * inv).astype(np.float32)
+    return e4m3_round(y.astype(F64)), (amax / np.float32(E4M3_MAX)).astype(np.float32).astype(F64)
+
+
+def attention_8bit(q, k, v, k_len: int | None = None, scale: float | None = None) -> np.ndarray:
+    """8-bit softmax attention of one sequence (q [Lq, n, d], k, v [Lk, n, d];
+    the first ``k_len`` keys valid). The scales of k and v are taken over all
+    Lk keys."""
+    q = np.asarray(q, F64)
+    k = np.asarray(k, F64)
+    v = np.asarray(v, F64)
+    Lq, n, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    qi, sq = quantize_int8(q, axes=(2,))           # [Lq, n, 1]
+    ki, sk = quantize_int8(k, axes=(0, 2))         # [1, n, 1]
+    vq, sv = quantize_fp8_axes(v, axes=(0,))       # [1, n, d]
+    kl = k.shape[0] if k_len is None else k_len
+    if kl == 0:
+        return np.zeros((Lq, n, d), F64)
+    ki, vq = ki[:kl], vq[:kl]
+    s = np.einsum("qnd,knd->nqk", qi, ki) * np.transpose(sq, (1, 0, 2)) * sk[0][:, :, None] * scale
+    p = np.exp(s - s.max(-1, keepdims=True))
+    pq = e4m3_round(p)
+    o = np.einsum("nqk,knd->qnd", pq, vq) * sv
+    return o / np.transpose(p.sum(-1, keepdims=True), (1, 0, 2))
+
+
+# --------------------------------------------------------------------------
 # The block ([WALK] WanAttentionBlock core-logic snippet; [DIGEST] shared
 # AdaLN MLP + per-block bias)
 # --------------------------------------------------------------------------
@@ -344,7 +406,7 @@ def self_attn_kv(x, e0, w, heads, grid, eps, theta=1e4, fp8=False):
 
 
 def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
-                       theta=1e4, kv=None, intermediates=None, fp8=False):
+                       theta=1e4, kv=None, intermediates=None, fp8=False, attn8=False):
     """Output of one WanAttentionBlock at the token rows ``rows`` of every
     sequence: [B, len(rows), D]. Follows the [WALK] block snippet:
 
@@ -363,6 +425,7 @@ def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
     ``intermediates`` (a dict) receives the per-branch outputs at those rows.
     ``fp8``: the ten projections (q, k, v, o, cross q, k, v, o, FFN 1 and 2)
     are FP8 linear layers (``linear_fp8``); everything else is unchanged.
+    ``attn8``: the self-attention is the 8-bit attention (``attention_8bit``).
     """
     linear = linear_fp8 if fp8 else _linear
     x = np.asarray(x, F64)
@@ -387,7 +450,7 @@ def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
         u = layer_norm(xb, eps) * (1.0 + m[b, 1]) + m[b, 0]
         q = rms_norm(linear(u, w["wq"], w["bq"]), w["gq"], eps).reshape(R, heads, d)
         q = rope_apply(q, grid, theta, positions=pos)
-        o = attention(q, k_all[b], v_all[b]).reshape(R, D)
+        o = (attention_8bit if attn8 else attention)(q, k_all[b], v_all[b]).reshape(R, D)
         y = linear(o, w["wo"], w["bo"])
         xb = xb + y * m[b, 2]
         inter["o_self"].append(o)
@@ -418,11 +481,12 @@ def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
 
 
 def block_forward(x, ctx, ctx_lens, e0, w, heads, grid, eps, theta=1e4,
-                  intermediates=None, fp8=False):
+                  intermediates=None, fp8=False, attn8=False):
     """Full block output [B, L, D] (all rows)."""
     L = np.asarray(x).shape[1]
     return block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps,
-                              np.arange(L), theta=theta, intermediates=intermediates, fp8=fp8)
+                              np.arange(L), theta=theta, intermediates=intermediates, fp8=fp8,
+                              attn8=attn8)
 
 
 # --------------------------------------------------------------------------
