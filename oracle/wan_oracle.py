@@ -303,11 +303,13 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
 # across key blocks). Readings where the page is silent: q is quantized per
 # token and head (scale amax/127 over the head's d values), k per head over
 # all keys of the sequence, v to e4m3 per head and channel over all keys
-# (the channel scale factors out of P V), and P = exp(s - max) in (0, 1] is
-# rounded to e4m3; the row normaliser is the exact sum of P. int8 codes are
-# round-half-even of x * (127 / amax), clamped to +-127, decided in fp32.
+# (the channel scale factors out of P V). Keys are taken in blocks of 128 in
+# order, FlashAttention style: each block's P = exp(s - m) uses the running
+# row max m after that block, is rounded to e4m3 for the P V product, and
+# the earlier sum and output are rescaled by exp(m_old - m); the row
+# normaliser sums the unrounded P. int8 codes are round-half-even of
+# x * (127 / amax), clamped to +-127, decided in fp32.
 # --------------------------------------------------------------------------
-
 I8_MAX = 127.0
 
 
@@ -335,10 +337,11 @@ def quantize_fp8_axes(x, axes):
     return e4m3_round(y.astype(F64)), (amax / np.float32(E4M3_MAX)).astype(np.float32).astype(F64)
 
 
-def attention_8bit(q, k, v, k_len: int | None = None, scale: float | None = None) -> np.ndarray:
+def attention_8bit(q, k, v, k_len: int | None = None, scale: float | None = None,
+                   block: int = 128) -> np.ndarray:
     """8-bit softmax attention of one sequence (q [Lq, n, d], k, v [Lk, n, d];
     the first ``k_len`` keys valid). The scales of k and v are taken over all
-    Lk keys."""
+    Lk keys; keys are visited in blocks of ``block``."""
     q = np.asarray(q, F64)
     k = np.asarray(k, F64)
     v = np.asarray(v, F64)
@@ -349,16 +352,22 @@ def attention_8bit(q, k, v, k_len: int | None = None, scale: float | None = None
     ki, sk = quantize_int8(k, axes=(0, 2))         # [1, n, 1]
     vq, sv = quantize_fp8_axes(v, axes=(0,))       # [1, n, d]
     kl = k.shape[0] if k_len is None else k_len
+    c = np.transpose(sq, (1, 0, 2)) * sk[0][:, :, None] * scale      # [n, Lq, 1]
+    m = np.full((n, Lq, 1), -np.inf)
+    l = np.zeros((n, Lq, 1))
+    o = np.zeros((n, Lq, d))
+    for j0 in range(0, kl, block):
+        j1 = min(j0 + block, kl)
+        s = np.einsum("qnd,knd->nqk", qi, ki[j0:j1]) * c            # exact integer products, scaled
+        m_new = np.maximum(m, s.max(-1, keepdims=True))
+        corr = np.exp(m - m_new)                                      # 0 on the first block
+        p = np.exp(s - m_new)
+        l = l * corr + p.sum(-1, keepdims=True)
+        o = o * corr + np.einsum("nqk,knd->nqd", e4m3_round(p), vq[j0:j1])
+        m = m_new
     if kl == 0:
         return np.zeros((Lq, n, d), F64)
-    ki, vq = ki[:kl], vq[:kl]
-    s = np.einsum("qnd,knd->nqk", qi, ki) * np.transpose(sq, (1, 0, 2)) * sk[0][:, :, None] * scale
-    p = np.exp(s - s.max(-1, keepdims=True))
-    pq = e4m3_round(p)
-    o = np.einsum("nqk,knd->qnd", pq, vq) * sv
-    return o / np.transpose(p.sum(-1, keepdims=True), (1, 0, 2))
-
-
+    return np.transpose(o / l, (1, 0, 2)) * sv
 # --------------------------------------------------------------------------
 # The block ([WALK] WanAttentionBlock core-logic snippet; [DIGEST] shared
 # AdaLN MLP + per-block bias)

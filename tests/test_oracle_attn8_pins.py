@@ -29,7 +29,7 @@ def test_quantize_int8_rules():
     assert s.shape == (1, 3, 1)
 
 
-def _exact_case(n=2, Lq=12, Lk=40, d=128, seed=1):
+def _exact_case(n=2, Lq=12, Lk=300, d=128, seed=1):
     """Inputs whose int8 / e4m3 quantization is exact (every scale is 1) and
     whose logits with scale ln 2 are small integers, so exp(s - max) is a
     power of two that e4m3 holds exactly."""
@@ -55,9 +55,14 @@ def test_attention_8bit_exact_when_quantization_is_identity():
     got = O.attention_8bit(q, k, v, scale=ln2)
     ref = O.attention(q, k, v, scale=ln2)
     assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
-    got = O.attention_8bit(q, k, v, k_len=17, scale=ln2)
-    ref = O.attention(q, k, v, k_len=17, scale=ln2)
-    assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
+    for kl in (17, 128, 129, 255):
+        got = O.attention_8bit(q, k, v, k_len=kl, scale=ln2)
+        ref = O.attention(q, k, v, k_len=kl, scale=ln2)
+        assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
+    # the key blocks only change where P is rounded: with every P a power of
+    # two the block size does not matter
+    assert np.abs(O.attention_8bit(q, k, v, scale=ln2, block=7) - O.attention_8bit(q, k, v, scale=ln2)).max() \
+        <= 1e-12 * np.abs(ref).max()
 
 
 def test_attention_8bit_scales_enter_where_they_should():
@@ -86,6 +91,9 @@ def test_attention_8bit_approximates_attention():
     err = np.linalg.norm(O.attention_8bit(q, k, v) - ref) / np.linalg.norm(ref)
     assert 1e-3 < err < 0.08
     assert not O.attention_8bit(q, k, v, k_len=0).any()
+    # one block holding every key: P is relative to the final row max
+    one = O.attention_8bit(q, k, v, block=256)
+    assert 1e-3 < np.linalg.norm(one - ref) / np.linalg.norm(ref) < 0.08
 
 
 def test_block_with_8bit_attention_close_to_fp8_block():
