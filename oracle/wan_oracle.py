@@ -304,11 +304,13 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
 # token and head (scale amax/127 over the head's d values), k per head over
 # all keys of the sequence, v to e4m3 per head and channel over all keys
 # (the channel scale factors out of P V). Keys are taken in blocks of 128 in
-# order, FlashAttention style: each block's P = exp(s - m) uses the running
-# row max m after that block, is rounded to e4m3 for the P V product, and
-# the earlier sum and output are rescaled by exp(m_old - m); the row
-# normaliser sums the unrounded P. int8 codes are round-half-even of
-# x * (127 / amax), clamped to +-127, decided in fp32.
+# order, FlashAttention style, in log2 units t = s log2(e): a row keeps a
+# frame F, the running max rounded up to a multiple of 8, raised after a
+# block whenever that block's max exceeds it (the earlier sum and output are
+# then rescaled by 2^(F_old - F)); the block's P = 2^(t - F + 8) lies in
+# (0, 2^8] and is rounded to e4m3 for the P V product; the row normaliser
+# sums the unrounded P. int8 codes are round-half-even of x * (127 / amax),
+# clamped to +-127, decided in fp32.
 # --------------------------------------------------------------------------
 I8_MAX = 127.0
 
@@ -352,19 +354,20 @@ def attention_8bit(q, k, v, k_len: int | None = None, scale: float | None = None
     ki, sk = quantize_int8(k, axes=(0, 2))         # [1, n, 1]
     vq, sv = quantize_fp8_axes(v, axes=(0,))       # [1, n, d]
     kl = k.shape[0] if k_len is None else k_len
-    c = np.transpose(sq, (1, 0, 2)) * sk[0][:, :, None] * scale      # [n, Lq, 1]
-    m = np.full((n, Lq, 1), -np.inf)
+    c = np.transpose(sq, (1, 0, 2)) * sk[0][:, :, None] * scale / math.log(2.0)    # [n, Lq, 1]
+    frame = np.full((n, Lq, 1), -np.inf)
     l = np.zeros((n, Lq, 1))
     o = np.zeros((n, Lq, d))
     for j0 in range(0, kl, block):
         j1 = min(j0 + block, kl)
-        s = np.einsum("qnd,knd->nqk", qi, ki[j0:j1]) * c            # exact integer products, scaled
-        m_new = np.maximum(m, s.max(-1, keepdims=True))
-        corr = np.exp(m - m_new)                                      # 0 on the first block
-        p = np.exp(s - m_new)
+        t = np.einsum("qnd,knd->nqk", qi, ki[j0:j1]) * c            # exact integer products, log2 units
+        tmax = t.max(-1, keepdims=True)
+        f_new = np.where(tmax > frame, 8.0 * np.ceil(tmax / 8.0), frame)
+        corr = np.exp2(frame - f_new)                                  # 0 on the first block
+        p = np.exp2(t - f_new + 8.0)
         l = l * corr + p.sum(-1, keepdims=True)
         o = o * corr + np.einsum("nqk,knd->nqd", e4m3_round(p), vq[j0:j1])
-        m = m_new
+        frame = f_new
     if kl == 0:
         return np.zeros((Lq, n, d), F64)
     return np.transpose(o / l, (1, 0, 2)) * sv
