@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--fp8", action="store_true",
                     help="FP8 GEMM mode of the blocks (e4m3 projections, bf16 attention); not the default")
+    ap.add_argument("--attn8", action="store_true",
+                    help="FP8 GEMMs and the 8-bit self-attention (int8 Q K^T, e4m3 P V); not the default")
     return ap.parse_args()
 
 
@@ -267,7 +269,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
     cfg = configs.get(args.config)
-    st = DenoiseStep(cfg, seed=1000 * rank, device=dev, fp8=args.fp8)
+    st = DenoiseStep(cfg, seed=1000 * rank, device=dev, fp8=args.fp8, attn8=args.attn8)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -352,33 +354,37 @@ def run_ours(args, rank, world, local_rank):
         avg_ms = attn_ms / attn_n
         tr = TRAFFIC.get("attn_self")
         traffic = None
-        if tr and tr.get("source_sha") == source_hash(*ATTN_SOURCES):
+        if tr and not args.attn8 and tr.get("source_sha") == source_hash(*ATTN_SOURCES):
             traffic = tr["bytes_per_launch"]
-        roofline = {"kernel": "attn_tc (self-attention, B=2, L=32760, 40 heads, d=128)",
+        apk = peak_sust * (2.0 if args.attn8 else 1.0)
+        roofline = {"kernel": ("attn8 (8-bit self-attention incl. its quantization passes" if args.attn8 else
+                               "attn_tc (self-attention") + ", B=2, L=32760, 40 heads, d=128)",
                     "bound": "tensor", "achieved": attn_flops_launch / (avg_ms * 1e-3) / 1e12,
-                    "peak": peak_sust, "unit": "TFLOP/s",
-                    "frac": attn_flops_launch / (avg_ms * 1e-3) / 1e12 / peak_sust,
-                    "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                    "peak": apk, "unit": "TFLOP/s",
+                    "frac": attn_flops_launch / (avg_ms * 1e-3) / 1e12 / apk,
+                    "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)"
+                                   + (" x 2 (8-bit / bf16 nominal ratio)" if args.attn8 else ""),
                     "traffic": traffic, "avg_launch_ms": avg_ms,
                     "algorithmic_flops_per_launch": attn_flops_launch}
     elif dom == "gemm_tc" and gemm_n:
-        gpk = peak_sust * (2.0 if args.fp8 else 1.0)
+        gpk = peak_sust * (2.0 if (args.fp8 or args.attn8) else 1.0)
         roofline = {"kernel": "gemm_tc (all block GEMMs)", "bound": "tensor", "achieved": gemm_tflops,
                     "peak": gpk, "unit": "TFLOP/s", "frac": gemm_tflops / gpk,
-                    "peak_source": f"{peak_src} bf16 sustained" + (" x 2 (fp8 / bf16 nominal ratio)" if args.fp8 else ""),
+                    "peak_source": f"{peak_src} bf16 sustained" + (" x 2 (fp8 / bf16 nominal ratio)" if (args.fp8 or args.attn8) else ""),
                     "traffic": None}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8 e4m3 GEMMs (per-token / per-tensor scales), bf16 attention" if args.fp8 else "bf16",
+        "dtype": ("fp8 e4m3 GEMMs, int8 QK^T / e4m3 PV self-attention" if args.attn8 else
+                  "fp8 e4m3 GEMMs (per-token / per-tensor scales), bf16 attention" if args.fp8 else "bf16"),
         "data": "synthetic",
         "impl": "ours",
         "config": workload_config(cfg, world),
         "attention_tflops": attn_tflops, "gemm_tflops": gemm_tflops,
         "attention_frac_of_2250": None if attn_tflops is None else attn_tflops / 2250.0,
         "gemm_frac_of_2250": None if gemm_tflops is None else gemm_tflops / 2250.0,
-        "gemm_frac_of_fp8_4500": None if (gemm_tflops is None or not args.fp8) else gemm_tflops / 4500.0,
+        "gemm_frac_of_fp8_4500": None if (gemm_tflops is None or not (args.fp8 or args.attn8)) else gemm_tflops / 4500.0,
         "kernel_ms_per_step": {k: v[1] / args.steps for k, v in prof.items() if v[0]},
         "gpu_launches": sum(v[0] for v in prof.values()),
         "roofline": roofline,
@@ -387,7 +393,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": e2e,
     }
     if world == 1 and not args.no_cpu_baseline:
-        ms, detail = OracleSample(cfg, seed=0, fp8=args.fp8).run()
+        ms, detail = OracleSample(cfg, seed=0, fp8=args.fp8 or args.attn8).run()
         line["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": cpu_cores(),
                                 "blas_threads": blas_threads(), "kind": "oracle", "sample": detail}
     print(json.dumps(line), flush=True)

@@ -52,6 +52,7 @@ typedef struct CUstream_st *wan_stream_t;
 #define WAN_F32  0
 #define WAN_BF16 1
 #define WAN_FP8  2   /* block mode: FP8 GEMMs, bf16 everything else (see wan_dims) */
+#define WAN_FP8_ATTN 3  /* block mode: WAN_FP8 plus the 8-bit self-attention      */
 
 /* Problem statement of one block call ([WALK]: grid sizes after the (1,2,2)
  * patch embedding, dim, heads, ffn_dim, text length, eps). */
@@ -73,7 +74,10 @@ typedef struct {
                        one scale each (wan_block_weights.w_scales) and every
                        projection's input is quantized to e4m3 per token
                        inside the block; the products run on the FP8 tensor
-                       cores and are accumulated in fp32.                    */
+                       cores and are accumulated in fp32.
+                       WAN_FP8_ATTN: WAN_FP8 with the self-attention run as
+                       wan_attention_8bit ([DIGEST] "8-bit FlashAttention");
+                       the cross-attention stays bf16.                       */
 } wan_dims;
 
 /* Parameters of one WanAttentionBlock ([WALK] block snippet). Pointers marked
@@ -131,7 +135,8 @@ size_t wan_block_workspace_bytes(const wan_dims *dims, int B);
 #define WAN_WS_A8     9  /* u8 [max(B*L*ffn, B*T*dim)] e4m3 codes of the last quantized GEMM input
                            (WAN_FP8 only; empty otherwise)                              */
 #define WAN_WS_ASCALE 10 /* f32 [max(B*L, B*T)] their per-row scales (WAN_FP8 only)       */
-#define WAN_WS_COUNT 11
+#define WAN_WS_ATTN8  11 /* scratch of the 8-bit self-attention (WAN_FP8_ATTN only)         */
+#define WAN_WS_COUNT 12
 /* Byte offset of buffer `which` inside the workspace, or (size_t)-1. */
 size_t wan_block_workspace_offset(const wan_dims *dims, int B, int which);
 
@@ -280,6 +285,25 @@ int wan_quantize_fp8(const void *src, int src_dtype, int rows, int cols, int per
  * Errors: WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED. */
 int wan_linear_fp8(int M, int N, int K, const uint8_t *a, const float *a_scale, const uint8_t *w,
                    const float *w_scale, const void *bias, float *out, wan_stream_t stream);
+
+/* wan_attention_8bit -- 8-bit flash attention ([DIGEST] inference-optimisation
+ * table, "8-bit FlashAttention": int8 for S = Q K^T, FP8 for O = P V, fp32
+ * accumulation across key blocks), non-causal, head_dim 128.
+ *   q, k, v   bf16 [B, Lq|Lk, heads, 128]; o out bf16 [B, Lq, heads, 128].
+ *   k_lens    as in wan_attention (device int32 [B] or NULL).
+ *   scale     logit scale; 0 for 1/sqrt(128).
+ *   workspace device scratch of wan_attention_8bit_workspace_bytes() bytes.
+ * Quantization inside the call (decisions in fp32): q to int8 per (token,
+ * head) with scale amax/127, k to int8 per (sequence, head) over all Lk keys,
+ * v to e4m3 per (sequence, head, channel) over all Lk keys (amax/448); int8
+ * codes are round-half-even of x * (127 / amax), clamped to +-127. S is
+ * accumulated exactly in int32, P = exp(S c - m) is rounded to e4m3 before
+ * the P V product (fp32 accumulation), the row sum uses the unrounded P.
+ * Errors: WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED (Lk == 0 included). */
+size_t wan_attention_8bit_workspace_bytes(int B, int heads, int Lq, int Lk);
+int wan_attention_8bit(int B, int heads, int Lq, int Lk, const void *q, const void *k, const void *v,
+                       void *o, const int *k_lens, float scale, void *workspace, size_t ws_bytes,
+                       wan_stream_t stream);
 
 /* wan_attention -- softmax attention, non-causal, every head
  * ([WALK] self-attention snippet: global window, key lengths).

@@ -65,6 +65,7 @@ struct WsLayout {
 };
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+static bool is_fp8(int dt) { return dt == WAN_FP8 || dt == WAN_FP8_ATTN; }
 
 static int check_dims(const wan_dims *d, int B) {
   if (!d) return set_error(WAN_EINVAL, "dims is NULL");
@@ -76,11 +77,11 @@ static int check_dims(const wan_dims *d, int B) {
   if (d->ffn_dim < 64 || d->ffn_dim % 64) return set_error(WAN_EINVAL, "ffn_dim %d must be a positive multiple of 64", d->ffn_dim);
   if (d->text_len < 0) return set_error(WAN_EINVAL, "text_len %d < 0", d->text_len);
   if (!(d->eps >= 0.f)) return set_error(WAN_EINVAL, "eps must be >= 0");
-  if (d->dtype != WAN_F32 && d->dtype != WAN_BF16 && d->dtype != WAN_FP8)
+  if (d->dtype != WAN_F32 && d->dtype != WAN_BF16 && !is_fp8(d->dtype))
     return set_error(WAN_EUNSUPPORTED, "dtype %d", d->dtype);
   const int hd = d->dim / d->heads;
   if (d->dtype != WAN_F32 && hd != 128) return set_error(WAN_EUNSUPPORTED, "bf16 / fp8 paths need head_dim 128 (got %d)", hd);
-  if (d->dtype == WAN_FP8 && (d->dim % 256 || d->ffn_dim % 128))
+  if (is_fp8(d->dtype) && (d->dim % 256 || d->ffn_dim % 128))
     return set_error(WAN_EUNSUPPORTED, "fp8 path needs dim %% 256 == 0 and ffn_dim %% 128 == 0");
   if (d->dtype == WAN_F32 && hd != 32 && hd != 64 && hd != 128)
     return set_error(WAN_EUNSUPPORTED, "fp32 path needs head_dim 32, 64 or 128 (got %d)", hd);
@@ -104,8 +105,9 @@ static WsLayout layout_of(const wan_dims *d, int B) {
       BL * Fh * es,           // H
       (size_t)B * 6 * D * 4,  // MOD
       (BL > (size_t)B * T ? BL : (size_t)B * T) * 4 * (D >= 256 ? D / 256 : 1) * 4,   // STATS: per-row partial sums of squares
-      d->dtype == WAN_FP8 ? (BL * Fh > (size_t)B * T * D ? BL * Fh : (size_t)B * T * D) : 0,   // A8
-      d->dtype == WAN_FP8 ? (BL > (size_t)B * T ? BL : (size_t)B * T) * 4 : 0,                // ASCALE
+      is_fp8(d->dtype) ? (BL * Fh > (size_t)B * T * D ? BL * Fh : (size_t)B * T * D) : 0,   // A8
+      is_fp8(d->dtype) ? (BL > (size_t)B * T ? BL : (size_t)B * T) * 4 : 0,                // ASCALE
+      d->dtype == WAN_FP8_ATTN && B > 0 ? attention_8bit_ws_bytes(B, d->heads, d->F * d->H * d->W, d->F * d->H * d->W) : 0,
   };
   size_t o = 0;
   for (int i = 0; i < WAN_WS_COUNT; ++i) {
@@ -173,7 +175,12 @@ static int block_forward_fp8(const wan_dims &d, int B, float *x, const void *ctx
     a.o = o; a.ldo = D; a.scale = scale;
     a.q_ss = stats; a.q_ss_stride = sstride; a.q_ss_parts = parts; a.q_ss_n = (float)D; a.q_ss_eps = d.eps;
     if (!attention_tc_supported(a)) return set_error(WAN_EUNSUPPORTED, "fp8 block: self-attention shape");
-    if ((rc = WAN_PROF(WAN_K_ATTN_SELF, s, attention_tc(a, s)))) return rc;
+    if (d.dtype == WAN_FP8_ATTN) {
+      if (!attention_8bit_supported(a)) return set_error(WAN_EUNSUPPORTED, "fp8 block: 8-bit self-attention shape");
+      if ((rc = WAN_PROF(WAN_K_ATTN_SELF, s, attention_8bit(a, ws + lay.off[WAN_WS_ATTN8], s)))) return rc;
+    } else if ((rc = WAN_PROF(WAN_K_ATTN_SELF, s, attention_tc(a, s)))) {
+      return rc;
+    }
   }
   if ((rc = quant_rows(o, BL, D))) return rc;
   {
@@ -291,7 +298,7 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
     if (!ptrs[i]) return set_error(WAN_EINVAL, "pointer argument #%zu is NULL", i);
     if (!aligned16(ptrs[i])) return set_error(WAN_EALIGN, "pointer argument #%zu not 16-byte aligned", i);
   }
-  if (dt == WAN_FP8) {
+  if (is_fp8(dt)) {
     if (!w->w_scales) return set_error(WAN_EINVAL, "WAN_FP8 needs w_scales");
     if (!aligned16(w->w_scales)) return set_error(WAN_EALIGN, "w_scales not 16-byte aligned");
   }
@@ -316,7 +323,7 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
 
   // m = modulation + e0  (shift, scale, gate, shift2, scale2, gate2)
   if ((rc = WAN_PROF(WAN_K_MISC, s, launch_mod_combine(w->modulation, e0, mod, B, D, s)))) return rc;
-  if (dt == WAN_FP8) return block_forward_fp8(d, B, x, ctx, ctx_lens, w, rope, ws, lay, mod, s);
+  if (is_fp8(dt)) return block_forward_fp8(d, B, x, ctx, ctx_lens, w, rope, ws, lay, mod, s);
 
   // ---- self-attention branch: x += m2 * Wo . Attn(RoPE(RMSNorm(q,k)), v)
   // bf16 tensor-core path: the QKV GEMM epilogue accumulates each row's sum of
@@ -467,6 +474,36 @@ int wan_linear_fp8(int M, int N, int K, const uint8_t *a, const float *a_scale, 
   if (!gemm_tc_supported(g)) return set_error(WAN_EUNSUPPORTED, "fp8 linear M=%d N=%d K=%d", M, N, K);
   cudaStream_t s = (cudaStream_t)stream;
   return WAN_PROF(WAN_K_GEMM_TC, s, gemm_tc(g, s));
+}
+
+size_t wan_attention_8bit_workspace_bytes(int B, int heads, int Lq, int Lk) {
+  if (B < 1 || heads < 1 || Lq < 1 || Lk < 1) return 0;
+  return attention_8bit_ws_bytes(B, heads, Lq, Lk);
+}
+
+int wan_attention_8bit(int B, int heads, int Lq, int Lk, const void *q, const void *k, const void *v,
+                       void *o, const int *k_lens, float scale, void *workspace, size_t ws_bytes,
+                       wan_stream_t stream) {
+  g_msg[0] = 0;
+  if (B < 0 || heads < 1 || Lq < 0 || Lk < 0) return set_error(WAN_EINVAL, "bad sizes");
+  if (B == 0 || Lq == 0) return WAN_OK;
+  if (Lk == 0) return set_error(WAN_EUNSUPPORTED, "8-bit attention needs Lk >= 1");
+  if ((long long)B * Lq * heads > INT_MAX / 32 || (long long)B * Lk * heads > INT_MAX / 32)
+    return set_error(WAN_EINVAL, "sizes too large");
+  const void *ps[] = {q, k, v, o, workspace};
+  for (const void *p : ps) {
+    if (!p) return set_error(WAN_EINVAL, "NULL pointer");
+    if (!aligned16(p)) return set_error(WAN_EALIGN, "pointer not 16-byte aligned");
+  }
+  if (k_lens && !aligned16(k_lens)) return set_error(WAN_EALIGN, "k_lens not 16-byte aligned");
+  if (ws_bytes < attention_8bit_ws_bytes(B, heads, Lq, Lk)) return set_error(WAN_EINVAL, "workspace too small");
+  AttnArgs a = {};
+  a.B = B; a.heads = heads; a.Lq = Lq; a.Lk = Lk; a.d = 128;
+  a.q = q; a.ldq = heads * 128; a.k = k; a.ldk = heads * 128; a.v = v; a.ldv = heads * 128;
+  a.o = o; a.ldo = heads * 128; a.k_lens = k_lens; a.scale = scale > 0.f ? scale : 1.0f / sqrtf(128.f);
+  if (!attention_8bit_supported(a)) return set_error(WAN_EUNSUPPORTED, "8-bit attention shape");
+  cudaStream_t s = (cudaStream_t)stream;
+  return WAN_PROF(WAN_K_ATTN_TC, s, attention_8bit(a, workspace, s));
 }
 
 int wan_attention(int B, int heads, int Lq, int Lk, int head_dim, int dtype, void *q, void *k,

@@ -148,6 +148,11 @@ struct AttnArgs {
   const float *q_ss; int q_ss_stride; int q_ss_parts; float q_ss_n; float q_ss_eps;
 };
 int attention_simt(const AttnArgs &a, int dtype, cudaStream_t s);
+// 8-bit attention (attn8.cu): bf16 q, k, v, o with head_dim 128; quantizes
+// into the workspace, then int8 Q K^T and e4m3 P V on the tensor cores
+size_t attention_8bit_ws_bytes(int B, int heads, int Lq, int Lk);
+bool attention_8bit_supported(const AttnArgs &a);
+int attention_8bit(const AttnArgs &a, void *workspace, cudaStream_t s);
 int attention_tc(const AttnArgs &a, cudaStream_t s);      // bf16, d = 128
 bool attention_tc_supported(const AttnArgs &a);
 

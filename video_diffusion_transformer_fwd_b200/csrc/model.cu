@@ -187,7 +187,7 @@ int wan_model_forward(const wan_model_dims *dims, int B, const float *latent, co
   if (ws_bytes < lay.total) return set_error(WAN_EINVAL, "workspace %zu bytes < %zu needed", ws_bytes, lay.total);
 
   cudaStream_t s = (cudaStream_t)stream;
-  const int dt = m.dtype == WAN_FP8 ? WAN_BF16 : m.dtype;    // embeddings and head stay bf16 in FP8 mode
+  const int dt = (m.dtype == WAN_FP8 || m.dtype == WAN_FP8_ATTN) ? WAN_BF16 : m.dtype;    // embeddings and head stay bf16 in FP8 mode
   const size_t es = dtype_size(dt);
   const int L = m.F * (m.H / 2) * (m.W / 2), BL = B * L, D = m.dim, T = m.text_len;
   char *ws = static_cast<char *>(workspace);

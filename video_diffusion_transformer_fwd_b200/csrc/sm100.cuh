@@ -162,6 +162,25 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "r"(z), "r"(z), "r"(z), "r"(z) : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem], kind::i8 (signed 8-bit, s32 accumulate).
+__device__ __forceinline__ void mma_ss_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem], kind::f8f6f4 (8-bit floats, f32 accumulate).
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
 // ---------------------------------------------------------------- CTA pairs (cta_group::2)
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -270,6 +289,12 @@ __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// kind::i8 instruction descriptor: s8 x s8 -> s32 (D format 2, A and B
+// format fields 1 = signed), M x N, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // 32 lanes x 32 consecutive 32-bit columns: thread t gets lane (base + t).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -321,6 +346,9 @@ int encode_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64
                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
 int encode_tmap_2d_f32(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows);
+int encode_tmap_3d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                      uint64_t batches, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
+                      uint32_t box_inner, uint32_t box_rows);
 int encode_tmap_3d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                         uint64_t batches, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
                         uint32_t box_inner, uint32_t box_rows);

@@ -53,16 +53,34 @@ int encode_tmap_2d_f32(CUtensorMap *map, const void *base, uint64_t inner, uint6
   return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, inner, rows, row_stride_bytes, box_inner, box_rows);
 }
 
+static int encode_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t rows,
+                     uint64_t batches, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
+                     uint32_t box_inner, uint32_t box_rows);
+
 int encode_tmap_3d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                         uint64_t batches, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
                         uint32_t box_inner, uint32_t box_rows) {
+  return encode_3d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, inner, rows, batches, row_stride_bytes,
+                   batch_stride_bytes, box_inner, box_rows);
+}
+
+int encode_tmap_3d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                      uint64_t batches, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
+                      uint32_t box_inner, uint32_t box_rows) {
+  return encode_3d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, rows, batches, row_stride_bytes,
+                   batch_stride_bytes, box_inner, box_rows);
+}
+
+static int encode_3d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t rows,
+                     uint64_t batches, uint64_t row_stride_bytes, uint64_t batch_stride_bytes,
+                     uint32_t box_inner, uint32_t box_rows) {
   auto enc = get_encode();
   if (!enc) return set_error(WAN_ECUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t gdim[3] = {inner, rows, batches};
   cuuint64_t gstride[2] = {row_stride_bytes, batch_stride_bytes};
   cuuint32_t box[3] = {box_inner, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), gdim, gstride, box,
+  CUresult r = enc(map, dt, 3, const_cast<void *>(base), gdim, gstride, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(WAN_ECUDA, "cuTensorMapEncodeTiled (3d) failed: %d", (int)r);

@@ -43,6 +43,7 @@ def main():
     ap.add_argument("what", choices=["attention", "block", "model"])
     ap.add_argument("--blocks", type=int, default=0)
     ap.add_argument("--fp8", action="store_true", help="block: FP8 GEMM mode")
+    ap.add_argument("--attn8", action="store_true", help="8-bit attention (block: with FP8 GEMMs)")
     ap.add_argument("--config", default="a14b-step")
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--L", type=int, default=16384)
@@ -57,9 +58,14 @@ def main():
         Lk = a.Lk or a.L
         q, k, v = synth.attention_inputs(a.B, a.L, Lk, a.heads, 128, "bf16", "cuda", 1)
         o = torch.empty_like(q)
-        ms, prof = _time(lambda: wan.attention(q, k, v, out=o), a.iters, a.warmup)
+        if a.attn8:
+            ws8 = torch.empty(wan.wan_attention_8bit_workspace_bytes(a.B, a.heads, a.L, Lk), dtype=torch.uint8,
+                              device="cuda")
+            ms, prof = _time(lambda: wan.attention_8bit(q, k, v, out=o, workspace=ws8), a.iters, a.warmup)
+        else:
+            ms, prof = _time(lambda: wan.attention(q, k, v, out=o), a.iters, a.warmup)
         flops = 4.0 * a.B * a.L * Lk * a.heads * 128
-        print(json.dumps({"what": "attention", "B": a.B, "Lq": a.L, "Lk": Lk, "heads": a.heads,
+        print(json.dumps({"what": "attention", "attn8": a.attn8, "B": a.B, "Lq": a.L, "Lk": Lk, "heads": a.heads,
                           "ms": ms, "tflops": flops / ms / 1e9, "kernels_ms": prof}))
         return
     cfg = configs.get(a.config)
@@ -71,8 +77,8 @@ def main():
     cfg = dataclasses.replace(cfg, batch=a.B)
     dims = wan.dims_of(cfg)
     w = synth.block_weights(cfg.dim, cfg.ffn_dim, cfg.dtype, "cuda", 0)
-    if a.fp8:
-        dims.dtype = wan.WAN_FP8
+    if a.fp8 or a.attn8:
+        dims.dtype = wan.WAN_FP8_ATTN if a.attn8 else wan.WAN_FP8
         w = wan.quantize_block_weights(w)
     acts = synth.block_activations(a.B, cfg.L, cfg.dim, cfg.text_len, cfg.dtype, "cuda", 100)
     rope = wan.rope_freqs(cfg.head_dim, 1024, cfg.theta)
@@ -80,7 +86,7 @@ def main():
     cw = wan.make_weights(w)
     ms, prof = _time(lambda: wan.block_forward(dims, acts["x"], acts["ctx"], acts["e0"], cw, rope, ws),
                      a.iters, a.warmup)
-    print(json.dumps({"what": "block", "config": cfg.name, "B": a.B, "L": cfg.L, "fp8": a.fp8, "ms": ms,
+    print(json.dumps({"what": "block", "config": cfg.name, "B": a.B, "L": cfg.L, "fp8": a.fp8, "attn8": a.attn8, "ms": ms,
                       "tflops": cfg.block_flops() / ms / 1e9,
                       "gemm_tflops": cfg.gemm_flops() / (prof.get("gemm_tc", 0) or float("nan")) / 1e9,
                       "attn_tflops": cfg.self_attn_flops() / (prof.get("attn_self", 0) or float("nan")) / 1e9,

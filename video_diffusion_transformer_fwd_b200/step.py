@@ -17,15 +17,16 @@ from .configs import BlockConfig
 
 class DenoiseStep:
     def __init__(self, cfg: BlockConfig, seed: int = 0, device: str = "cuda", weights=None,
-                 fp8: bool = False):
+                 fp8: bool = False, attn8: bool = False):
         """``fp8``: the blocks run their projections as FP8 GEMMs (the bf16
-        weights are quantized per tensor once, here)."""
+        weights are quantized per tensor once, here); ``attn8`` also runs the
+        self-attention as the 8-bit attention."""
         self.cfg = cfg
         self.dims = wan.dims_of(cfg)
         self.device = device
         self.weights = weights if weights is not None else synth.step_weights(cfg, device, seed)
-        if fp8:
-            self.dims.dtype = wan.WAN_FP8
+        if fp8 or attn8:
+            self.dims.dtype = wan.WAN_FP8_ATTN if attn8 else wan.WAN_FP8
             self.weights = [wan.quantize_block_weights(w) for w in self.weights]
         self.cweights = [wan.make_weights(w) for w in self.weights]
         acts = synth.block_activations(2, cfg.L, cfg.dim, cfg.text_len, cfg.dtype, device,

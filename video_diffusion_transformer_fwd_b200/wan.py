@@ -15,10 +15,10 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libwan.so")
 
 WAN_OK, WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED, WAN_ECUDA, WAN_ETIMEOUT = 0, -1, -2, -3, -4, -5
-WAN_F32, WAN_BF16, WAN_FP8 = 0, 1, 2
+WAN_F32, WAN_BF16, WAN_FP8, WAN_FP8_ATTN = 0, 1, 2, 3
 WAN_NOALLOC_WORKSPACE_BYTES = 16 << 20
 (WAN_WS_ACT, WAN_WS_QKV, WAN_WS_O, WAN_WS_QC, WAN_WS_KVC, WAN_WS_OC, WAN_WS_H, WAN_WS_MOD,
- WAN_WS_STATS, WAN_WS_A8, WAN_WS_ASCALE) = range(11)
+ WAN_WS_STATS, WAN_WS_A8, WAN_WS_ASCALE, WAN_WS_ATTN8) = range(12)
 (WAN_K_GEMM_TC, WAN_K_GEMM_SIMT, WAN_K_ATTN_SELF, WAN_K_ATTN_CROSS, WAN_K_ATTN_SIMT, WAN_K_LAYERNORM,
  WAN_K_QKNORM_ROPE, WAN_K_EULER, WAN_K_MISC, WAN_K_ATTN_TC, WAN_K_MODEL, WAN_K_QUANT) = range(12)
 WAN_K_COUNT = 12
@@ -90,6 +90,9 @@ _SIGS = {
     "wan_model_workspace_bytes": (_sz, [ctypes.POINTER(wan_model_dims), _c_int]),
     "wan_quantize_fp8": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "wan_linear_fp8": (_c_int, [_c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "wan_attention_8bit_workspace_bytes": (_sz, [_c_int, _c_int, _c_int, _c_int]),
+    "wan_attention_8bit": (_c_int, [_c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
+                                    _vp, _sz, _vp]),
     "wan_model_forward": (_c_int, [ctypes.POINTER(wan_model_dims), _c_int, _vp, _vp, _vp, _vp,
                                    ctypes.POINTER(wan_model_weights),
                                    ctypes.POINTER(wan_block_weights), _c_int, _vp, _c_int, _vp,
@@ -185,6 +188,15 @@ def wan_linear_fp8(M, N, K, a, a_scale, w, w_scale, bias, out, stream):
     return load().wan_linear_fp8(M, N, K, a, a_scale, w, w_scale, bias, out, stream)
 
 
+def wan_attention_8bit_workspace_bytes(B, heads, Lq, Lk):
+    return load().wan_attention_8bit_workspace_bytes(B, heads, Lq, Lk)
+
+
+def wan_attention_8bit(B, heads, Lq, Lk, q, k, v, o, k_lens, scale, workspace, ws_bytes, stream):
+    return load().wan_attention_8bit(B, heads, Lq, Lk, q, k, v, o, k_lens, scale, workspace, ws_bytes,
+                                     stream)
+
+
 def wan_device_status(stream):
     return load().wan_device_status(stream)
 
@@ -238,7 +250,7 @@ def dtype_code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-DTYPE_CODES = {"bf16": WAN_BF16, "f32": WAN_F32, "fp8": WAN_FP8}
+DTYPE_CODES = {"bf16": WAN_BF16, "f32": WAN_F32, "fp8": WAN_FP8, "fp8attn": WAN_FP8_ATTN}
 
 
 def make_dims(F, H, W, dim, heads, ffn_dim, text_len, eps=1e-6, dtype="bf16") -> wan_dims:
@@ -352,6 +364,20 @@ def attention(q, k, v, k_lens=None, scale=0.0, grid=None, rope=None, out=None, s
     check(wan_attention(B, n, Lq, Lk, d, dtype_code(q), q.data_ptr(), k.data_ptr(), v.data_ptr(),
                         o.data_ptr(), _ptr(k_lens), scale, grid, _ptr(rope),
                         0 if rope is None else rope.shape[0], _stream(stream)))
+    return o
+
+
+def attention_8bit(q, k, v, k_lens=None, scale=0.0, out=None, workspace=None, stream=None):
+    """8-bit attention: q [B, Lq, n, 128], k / v [B, Lk, n, 128] bf16."""
+    torch = _torch()
+    B, Lq, n, d = q.shape
+    Lk = k.shape[1]
+    o = torch.empty_like(q) if out is None else out
+    if workspace is None:
+        workspace = torch.empty(max(wan_attention_8bit_workspace_bytes(B, n, Lq, Lk), 1), dtype=torch.uint8,
+                                device=q.device)
+    check(wan_attention_8bit(B, n, Lq, Lk, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), _ptr(k_lens),
+                             scale, workspace.data_ptr(), workspace.numel(), _stream(stream)))
     return o
 
 
