@@ -397,8 +397,20 @@ def block_param_count(dim: int, ffn_dim: int, biases: bool = True) -> int:
 
 
 def _mod(w, e0):
-    # e = (modulation + e0).chunk(6): shift, scale, gate, shift2, scale2, gate2
-    return np.asarray(w["modulation"], F64)[None] + np.asarray(e0, F64)   # [B, 6, D]
+    """e = (modulation + e0).chunk(6): shift, scale, gate, shift2, scale2,
+    gate2. e0 is [B, 6, D] (one timestep per sequence) or [B, L, 6, D] (one
+    per token: [WALK] time-projection snippet, ``unflatten(0, (bt, seq_len))``)."""
+    e0 = np.asarray(e0, F64)
+    mod = np.asarray(w["modulation"], F64)
+    return (mod[None] if e0.ndim == 3 else mod[None, None]) + e0
+
+
+def _chunk(m, k, b=None, rows=None):
+    """Chunk k of the modulation for every row: [B, L or 1, D] (b None) or
+    [R or 1, D] for sequence b at ``rows``."""
+    if m.ndim == 3:                                   # per sequence
+        return m[:, k, None, :] if b is None else m[b, k][None]
+    return m[:, :, k, :] if b is None else m[b, rows, k]
 
 
 def self_attn_kv(x, e0, w, heads, grid, eps, theta=1e4, fp8=False):
@@ -410,7 +422,7 @@ def self_attn_kv(x, e0, w, heads, grid, eps, theta=1e4, fp8=False):
     B, L, D = x.shape
     d = D // heads
     m = _mod(w, e0)
-    u = layer_norm(x, eps) * (1.0 + m[:, 1, None, :]) + m[:, 0, None, :]
+    u = layer_norm(x, eps) * (1.0 + _chunk(m, 1)) + _chunk(m, 0)
     k = rms_norm(linear(u, w["wk"], w["bk"]), w["gk"], eps).reshape(B, L, heads, d)
     v = linear(u, w["wv"], w["bv"]).reshape(B, L, heads, d)
     k = np.stack([rope_apply(k[b], grid, theta) for b in range(B)])
@@ -459,12 +471,12 @@ def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
     for b in range(B):
         xb = xr[b]
         # self-attention branch
-        u = layer_norm(xb, eps) * (1.0 + m[b, 1]) + m[b, 0]
+        u = layer_norm(xb, eps) * (1.0 + _chunk(m, 1, b, rows)) + _chunk(m, 0, b, rows)
         q = rms_norm(linear(u, w["wq"], w["bq"]), w["gq"], eps).reshape(R, heads, d)
         q = rope_apply(q, grid, theta, positions=pos)
         o = (attention_8bit if attn8 else attention)(q, k_all[b], v_all[b]).reshape(R, D)
         y = linear(o, w["wo"], w["bo"])
-        xb = xb + y * m[b, 2]
+        xb = xb + y * _chunk(m, 2, b, rows)
         inter["o_self"].append(o)
         inter["y_self"].append(y)
         # cross-attention branch
@@ -479,10 +491,10 @@ def block_forward_rows(x, ctx, ctx_lens, e0, w, heads, grid, eps, rows,
         inter["o_cross"].append(oc)
         inter["y_cross"].append(yc)
         # FFN branch
-        a2 = layer_norm(xb, eps) * (1.0 + m[b, 4]) + m[b, 3]
+        a2 = layer_norm(xb, eps) * (1.0 + _chunk(m, 4, b, rows)) + _chunk(m, 3, b, rows)
         h = gelu_tanh(linear(a2, w["w1"], w["b1"]))
         yf = linear(h, w["w2"], w["b2"])
-        xb = xb + yf * m[b, 5]
+        xb = xb + yf * _chunk(m, 5, b, rows)
         inter["h"].append(h)
         inter["y_ffn"].append(yf)
         out[b] = xb
@@ -577,10 +589,11 @@ def silu(z):
 def time_embed(t, mw, freq_dim=256):
     """e = Linear(SiLU(Linear(sinusoid(t)))) and e0 = Linear(SiLU(e)) as
     [B, 6, dim] ([WALK] structure and time-projection snippets)."""
+    shape = np.shape(t)                                # [B] or [B, L] (one timestep per token)
     s = sinusoidal_embedding(freq_dim, t)
     e = linear(silu(linear(s, mw["time_w1"], mw["time_b1"])), mw["time_w2"], mw["time_b2"])
     e0 = linear(silu(e), mw["proj_w"], mw["proj_b"])
-    return e, e0.reshape(e.shape[0], 6, -1)
+    return e.reshape(shape + (-1,)), e0.reshape(shape + (6, -1))
 
 
 def text_embed(ctx_raw, mw):
@@ -605,9 +618,15 @@ def patch_embed(latent, mw):
 
 
 def head(x, e, mw, eps):
-    """LN(x) (1 + m1) + m0 with m = head_modulation + e, then Linear."""
-    m = np.asarray(mw["head_mod"], F64)[None] + np.asarray(e, F64)[:, None, :]   # [B, 2, dim]
-    u = layer_norm(x, eps) * (1.0 + m[:, 1, None, :]) + m[:, 0, None, :]
+    """LN(x) (1 + m1) + m0 with m = head_modulation + e, then Linear; e is
+    [B, dim] or, with per-token timesteps, [B, L, dim]."""
+    e = np.asarray(e, F64)
+    hm = np.asarray(mw["head_mod"], F64)
+    if e.ndim == 2:
+        m0, m1 = (hm[0][None] + e)[:, None, :], (hm[1][None] + e)[:, None, :]
+    else:
+        m0, m1 = hm[0] + e, hm[1] + e
+    u = layer_norm(x, eps) * (1.0 + m1) + m0
     return linear(u, mw["head_w"], mw["head_b"])
 
 
@@ -623,7 +642,8 @@ def unpatchify(tokens, grid, channels):
 
 def model_forward(latent, t, ctx_raw, ctx_lens, mw, blocks, heads, eps, theta=1e4, freq_dim=256):
     """WanModel forward on latents ([WALK] forward snippet): patch embedding,
-    flatten, time and text embeddings, the block stack, head, unpatchify."""
+    flatten, time and text embeddings, the block stack, head, unpatchify.
+    t is [B] or [B, L] (a timestep per token, L = F (H/2) (W/2))."""
     latent = np.asarray(latent, F64)
     B, C, Fl, Hl, Wl = latent.shape
     grid = (Fl, Hl // 2, Wl // 2)
