@@ -78,6 +78,10 @@ typedef struct {
                        WAN_FP8_ATTN: WAN_FP8 with the self-attention run as
                        wan_attention_8bit ([DIGEST] "8-bit FlashAttention");
                        the cross-attention stays bf16.                       */
+  int e0_per_token; /* 0: e0 is [B, 6, dim] (one timestep per sequence);
+                       1: e0 is [B, L, 6, dim], one timestep per token
+                       ([WALK] time-projection snippet: the embedding is
+                       unflattened to (batch, seq_len); TI2V)                */
 } wan_dims;
 
 /* Parameters of one WanAttentionBlock ([WALK] block snippet). Pointers marked
@@ -160,7 +164,8 @@ size_t wan_block_workspace_offset(const wan_dims *dims, int B, int which);
  *   ctx       (dt) [B, T, dim] projected text tokens.
  *   ctx_lens  device int32 [B] valid text tokens (0..T), or NULL (all T).
  *   e0        float32 [B, 6, dim] time projection (shift, scale, gate,
- *             shift2, scale2, gate2), shared by all blocks of a step.
+ *             shift2, scale2, gate2), shared by all blocks of a step; with
+ *             dims->e0_per_token, [B, L, 6, dim], one per token.
  *   w         block parameters (host struct of device pointers).
  *   rope      table from wan_rope_freqs(head_dim, max_pos >= max(F,H,W)).
  *   rope_max_pos  rows in that table.
@@ -223,6 +228,8 @@ typedef struct {
   int dtype;            /* WAN_F32 | WAN_BF16 | WAN_FP8, as in wan_dims; with
                            WAN_FP8 the blocks run their FP8 GEMMs and the
                            embeddings and head are bf16                           */
+  int t_per_token;      /* 0: t is [B]; 1: t is [B, L] (L = F (H/2) (W/2)), one
+                           timestep per token; the blocks then get e0 per token */
 } wan_model_dims;
 
 /* (dt) = wan_model_dims.dtype; others float32. */

@@ -67,6 +67,27 @@ struct WsLayout {
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 static bool is_fp8(int dt) { return dt == WAN_FP8 || dt == WAN_FP8_ATTN; }
 
+// Modulation source of a block call: the combined [B, 6, D] (one timestep per
+// sequence) or the caller's per-token e0 [B*L, 6, D] plus the block's
+// modulation, added where they are read.
+struct ModSrc {
+  bool ptok;
+  const float *e0, *mod, *modulation;
+  int L, D;
+};
+static LnMod ln_of(const ModSrc &m, int shift_chunk, int scale_chunk) {
+  return m.ptok ? ln_mod_tok(m.e0, m.modulation, m.D, shift_chunk, scale_chunk)
+                : ln_mod_seq(m.mod, m.L, m.D, shift_chunk, scale_chunk);
+}
+static void gate_of(const ModSrc &m, GemmArgs &g, int chunk) {
+  g.gate_stride = 6 * m.D;
+  if (m.ptok) {
+    g.gate = m.e0 + chunk * m.D; g.rows_per_gate = 1; g.gate_bias = m.modulation + chunk * m.D;
+  } else {
+    g.gate = m.mod + chunk * m.D; g.rows_per_gate = m.L;
+  }
+}
+
 static int check_dims(const wan_dims *d, int B) {
   if (!d) return set_error(WAN_EINVAL, "dims is NULL");
   if (B < 0) return set_error(WAN_EINVAL, "B=%d < 0", B);
@@ -77,6 +98,7 @@ static int check_dims(const wan_dims *d, int B) {
   if (d->ffn_dim < 64 || d->ffn_dim % 64) return set_error(WAN_EINVAL, "ffn_dim %d must be a positive multiple of 64", d->ffn_dim);
   if (d->text_len < 0) return set_error(WAN_EINVAL, "text_len %d < 0", d->text_len);
   if (!(d->eps >= 0.f)) return set_error(WAN_EINVAL, "eps must be >= 0");
+  if (d->e0_per_token != 0 && d->e0_per_token != 1) return set_error(WAN_EINVAL, "e0_per_token must be 0 or 1");
   if (d->dtype != WAN_F32 && d->dtype != WAN_BF16 && !is_fp8(d->dtype))
     return set_error(WAN_EUNSUPPORTED, "dtype %d", d->dtype);
   const int hd = d->dim / d->heads;
@@ -128,7 +150,7 @@ static WsLayout layout_of(const wan_dims *d, int B) {
 // scales before the bias, q/k-norm, GELU or gated residual.
 static int block_forward_fp8(const wan_dims &d, int B, float *x, const void *ctx, const int *ctx_lens,
                              const wan_block_weights *w, const float *rope, char *ws, const WsLayout &lay,
-                             const float *mod, cudaStream_t s) {
+                             const ModSrc &ms, cudaStream_t s) {
   const int L = d.F * d.H * d.W, D = d.dim, T = d.text_len, Fh = d.ffn_dim, hd = D / d.heads, BL = B * L;
   const size_t es = 2;
   char *qkv = ws + lay.off[WAN_WS_QKV];
@@ -154,7 +176,7 @@ static int block_forward_fp8(const wan_dims &d, int B, float *x, const void *ctx
   };
 
   // ---- self-attention
-  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod_fp8(x, a8, asc, BL, D, L, mod, 0, 1, nullptr, nullptr, d.eps, s)))) return rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod_fp8(x, a8, asc, BL, D, ln_of(ms, 0, 1), nullptr, nullptr, d.eps, s)))) return rc;
   {
     GemmArgs g = {};
     g.M = BL; g.N = 3 * D; g.K = D;
@@ -187,12 +209,13 @@ static int block_forward_fp8(const wan_dims &d, int B, float *x, const void *ctx
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = D; g.Bseg[0] = w->wo; g.bias[0] = w->bo; g.b_scale[0] = wsc + 3;
     g.segN = D; g.nseg = 1;
-    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = mod + 2 * D; g.gate_stride = 6 * D; g.rows_per_gate = L;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D;
+    gate_of(ms, g, 2);
     if ((rc = gemm8(g))) return rc;
   }
 
   // ---- cross-attention (ungated)
-  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod_fp8(x, a8, asc, BL, D, L, nullptr, 0, 0, w->g3, w->b3, d.eps, s)))) return rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod_fp8(x, a8, asc, BL, D, LnMod{}, w->g3, w->b3, d.eps, s)))) return rc;
   {
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = D; g.Bseg[0] = w->cwq; g.bias[0] = w->cbq; g.b_scale[0] = wsc + 4;
@@ -230,7 +253,7 @@ static int block_forward_fp8(const wan_dims &d, int B, float *x, const void *ctx
   }
 
   // ---- FFN
-  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod_fp8(x, a8, asc, BL, D, L, mod, 3, 4, nullptr, nullptr, d.eps, s)))) return rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod_fp8(x, a8, asc, BL, D, ln_of(ms, 3, 4), nullptr, nullptr, d.eps, s)))) return rc;
   {
     GemmArgs g = {};
     g.M = BL; g.N = Fh; g.K = D; g.Bseg[0] = w->w1; g.bias[0] = w->b1; g.b_scale[0] = wsc + 8;
@@ -242,7 +265,8 @@ static int block_forward_fp8(const wan_dims &d, int B, float *x, const void *ctx
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = Fh; g.Bseg[0] = w->w2; g.bias[0] = w->b2; g.b_scale[0] = wsc + 9;
     g.segN = D; g.nseg = 1;
-    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = mod + 5 * D; g.gate_stride = 6 * D; g.rows_per_gate = L;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D;
+    gate_of(ms, g, 5);
     if ((rc = gemm8(g))) return rc;
   }
   return WAN_OK;
@@ -322,8 +346,9 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
   const int BL = B * L;
 
   // m = modulation + e0  (shift, scale, gate, shift2, scale2, gate2)
-  if ((rc = WAN_PROF(WAN_K_MISC, s, launch_mod_combine(w->modulation, e0, mod, B, D, s)))) return rc;
-  if (is_fp8(dt)) return block_forward_fp8(d, B, x, ctx, ctx_lens, w, rope, ws, lay, mod, s);
+  const ModSrc ms{d.e0_per_token != 0, e0, mod, w->modulation, L, D};
+  if (!ms.ptok && (rc = WAN_PROF(WAN_K_MISC, s, launch_mod_combine(w->modulation, e0, mod, B, D, s)))) return rc;
+  if (is_fp8(dt)) return block_forward_fp8(d, B, x, ctx, ctx_lens, w, rope, ws, lay, ms, s);
 
   // ---- self-attention branch: x += m2 * Wo . Attn(RoPE(RMSNorm(q,k)), v)
   // bf16 tensor-core path: the QKV GEMM epilogue accumulates each row's sum of
@@ -348,7 +373,7 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
   aself.o = o; aself.ldo = D; aself.k_lens = nullptr; aself.scale = 1.0f / sqrtf((float)hd);
   const bool fused = dt == WAN_BF16 && gemm_tc_supported(gqkv) && attention_tc_supported(aself);
 
-  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, L, mod, 0, 1, nullptr, nullptr, d.eps, s)))) return rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, ln_of(ms, 0, 1), nullptr, nullptr, d.eps, s)))) return rc;
   if (fused) {
     if ((rc = run_gemm(gqkv, dt, s))) return rc;
     if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_scale_rows(qkv + D * es, BL, 3 * D, D, stats + parts, sstride, parts, d.eps, s)))) return rc;
@@ -364,12 +389,13 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = D; g.A = o; g.lda = D;
     g.Bseg[0] = w->wo; g.bias[0] = w->bo; g.segN = D; g.nseg = 1;
-    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = mod + 2 * D; g.gate_stride = 6 * D; g.rows_per_gate = L;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D;
+    gate_of(ms, g, 2);
     if ((rc = run_gemm(g, dt, s))) return rc;
   }
 
   // ---- cross-attention branch (ungated): x += Wco . Attn(q(norm3 x), k(ctx), v(ctx))
-  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, L, nullptr, 0, 0, w->g3, w->b3, d.eps, s)))) return rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, LnMod{}, w->g3, w->b3, d.eps, s)))) return rc;
   {
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = D; g.A = act; g.lda = D;
@@ -415,7 +441,7 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
   }
 
   // ---- FFN branch: x += m5 * W2 . gelu_tanh(W1 . (LN(x)(1 + m4) + m3))
-  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, L, mod, 3, 4, nullptr, nullptr, d.eps, s)))) return rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, ln_of(ms, 3, 4), nullptr, nullptr, d.eps, s)))) return rc;
   {
     GemmArgs g = {};
     g.M = BL; g.N = Fh; g.K = D; g.A = act; g.lda = D;
@@ -427,7 +453,8 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
     GemmArgs g = {};
     g.M = BL; g.N = D; g.K = Fh; g.A = hbuf; g.lda = Fh;
     g.Bseg[0] = w->w2; g.bias[0] = w->b2; g.segN = D; g.nseg = 1;
-    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = mod + 5 * D; g.gate_stride = 6 * D; g.rows_per_gate = L;
+    g.epi = EPI_RESID; g.X = x; g.ldx = D;
+    gate_of(ms, g, 5);
     if ((rc = run_gemm(g, dt, s))) return rc;
   }
   return WAN_OK;

@@ -118,6 +118,7 @@ struct GemmArgs {
   void *C; int ldc;
   float *X; int ldx;
   const float *gate; int gate_stride; int rows_per_gate;
+  const float *gate_bias;  // optional [N]: g = gate[...] + gate_bias[n] (per-token modulation)
   int x_store;            // EPI_RESID: x = g * y (overwrite) instead of x += g * y
   int fp8;                // A and B are e4m3 codes: y = (A B^T) a_scale[m] b_scale[seg] + bias
   const float *a_scale;   // [M] (device)
@@ -161,12 +162,25 @@ int launch_mod_combine(const float *modulation, const float *e0, float *mod, int
                        cudaStream_t s);
 // out[r] = LN(x[r]) * (1 + mod[b][scale_chunk]) + mod[b][shift_chunk]     (affine == NULL)
 // out[r] = LN(x[r]) * g + beta                                            (affine gain g)
-int launch_layernorm_mod(const float *x, void *out, int dtype, int rows, int D, int rows_per_b,
-                         const float *mod, int shift_chunk, int scale_chunk,
+// Where a LayerNorm row finds its modulation: shift = mod[(row / rows_div) *
+// row_stride + shift_off + c] (+ bias[bias_shift_off + c] when bias is set),
+// likewise scale. mod == nullptr: the affine g, beta instead.
+struct LnMod {
+  const float *mod; int rows_div; size_t row_stride; int shift_off, scale_off;
+  const float *bias; int bias_shift_off, bias_scale_off;
+};
+// chunks of a combined [B, 6, D] modulation, L rows per sequence
+inline LnMod ln_mod_seq(const float *mod, int L, int D, int shift_chunk, int scale_chunk) {
+  return LnMod{mod, L, (size_t)6 * D, shift_chunk * D, scale_chunk * D, nullptr, 0, 0};
+}
+// chunks of a per-token e0 [rows, 6, D] plus the block's modulation [6, D]
+inline LnMod ln_mod_tok(const float *e0, const float *modulation, int D, int shift_chunk, int scale_chunk) {
+  return LnMod{e0, 1, (size_t)6 * D, shift_chunk * D, scale_chunk * D, modulation, shift_chunk * D, scale_chunk * D};
+}
+int launch_layernorm_mod(const float *x, void *out, int dtype, int rows, int D, const LnMod &m,
                          const float *g, const float *beta, float eps, cudaStream_t s);
 // the same with the output quantized per row to e4m3 codes q and scales row_scale
-int launch_layernorm_mod_fp8(const float *x, uint8_t *q, float *row_scale, int rows, int D, int rows_per_b,
-                             const float *mod, int shift_chunk, int scale_chunk,
+int launch_layernorm_mod_fp8(const float *x, uint8_t *q, float *row_scale, int rows, int D, const LnMod &m,
                              const float *g, const float *beta, float eps, cudaStream_t s);
 // e4m3 quantization per row (src rows ld elements apart) or per tensor (n elements)
 int launch_quant_rows(const void *src, int dtype, size_t ld, int rows, int cols, uint8_t *q, float *scale,

@@ -213,8 +213,7 @@ constexpr int LN_MAXV = 8;          // float4 per thread: D <= 8192
 // scale (written to row_scale), the input of an FP8 GEMM.
 template <typename OutT>
 __global__ void __launch_bounds__(LN_THREADS)
-layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int D, int rows_per_b,
-                     const float *__restrict__ mod, int shift_chunk, int scale_chunk,
+layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int D, const LnMod md,
                      const float *__restrict__ g, const float *__restrict__ beta, float eps,
                      float *__restrict__ row_scale) {
   __shared__ float red[32];
@@ -243,11 +242,15 @@ layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int D,
   }
   const float var = block_sum(ss, red) / (float)D;
   const float rstd = 1.0f / sqrtf(var + eps);
-  const float *mshift = nullptr, *mscale = nullptr;
-  if (g == nullptr) {
-    const int b = row / rows_per_b;
-    mshift = mod + ((size_t)b * 6 + shift_chunk) * D;
-    mscale = mod + ((size_t)b * 6 + scale_chunk) * D;
+  const float *mshift = nullptr, *mscale = nullptr, *bshift = nullptr, *bscale = nullptr;
+  if (md.mod) {
+    const float *mrow = md.mod + (size_t)(row / md.rows_div) * md.row_stride;
+    mshift = mrow + md.shift_off;
+    mscale = mrow + md.scale_off;
+    if (md.bias) {
+      bshift = md.bias + md.bias_shift_off;
+      bscale = md.bias + md.bias_scale_off;
+    }
   }
   OutT *orow = out + (size_t)row * D;
   float amax = 0.f;
@@ -258,8 +261,13 @@ layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int D,
       float4 u = make_float4((v[i].x - mean) * rstd, (v[i].y - mean) * rstd,
                              (v[i].z - mean) * rstd, (v[i].w - mean) * rstd);
       float4 a, b;
-      if (g == nullptr) {
-        const float4 sc = load4(mscale + 4 * c), sh = load4(mshift + 4 * c);
+      if (md.mod) {
+        float4 sc = load4(mscale + 4 * c), sh = load4(mshift + 4 * c);
+        if (bshift) {
+          const float4 bs = load4(bscale + 4 * c), bh = load4(bshift + 4 * c);
+          sc = make_float4(sc.x + bs.x, sc.y + bs.y, sc.z + bs.z, sc.w + bs.w);
+          sh = make_float4(sh.x + bh.x, sh.y + bh.y, sh.z + bh.z, sh.w + bh.w);
+        }
         a = make_float4(1.f + sc.x, 1.f + sc.y, 1.f + sc.z, 1.f + sc.w);
         b = sh;
       } else {
@@ -291,28 +299,23 @@ layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int D,
   }
 }
 
-int launch_layernorm_mod(const float *x, void *out, int dtype, int rows, int D, int rows_per_b,
-                         const float *mod, int shift_chunk, int scale_chunk,
+int launch_layernorm_mod(const float *x, void *out, int dtype, int rows, int D, const LnMod &m,
                          const float *g, const float *beta, float eps, cudaStream_t s) {
   if (D % 4 || D > 4 * LN_MAXV * LN_THREADS) return set_error(WAN_EUNSUPPORTED, "layernorm: D=%d", D);
   if (rows == 0) return WAN_OK;
   if (dtype == WAN_BF16)
-    layernorm_mod_kernel<__nv_bfloat16><<<rows, LN_THREADS, 0, s>>>(
-        x, (__nv_bfloat16 *)out, D, rows_per_b, mod, shift_chunk, scale_chunk, g, beta, eps, nullptr);
+    layernorm_mod_kernel<__nv_bfloat16><<<rows, LN_THREADS, 0, s>>>(x, (__nv_bfloat16 *)out, D, m, g, beta, eps, nullptr);
   else
-    layernorm_mod_kernel<float><<<rows, LN_THREADS, 0, s>>>(
-        x, (float *)out, D, rows_per_b, mod, shift_chunk, scale_chunk, g, beta, eps, nullptr);
+    layernorm_mod_kernel<float><<<rows, LN_THREADS, 0, s>>>(x, (float *)out, D, m, g, beta, eps, nullptr);
   WAN_CHECK_LAUNCH("layernorm_mod");
   return WAN_OK;
 }
 
-int launch_layernorm_mod_fp8(const float *x, uint8_t *q, float *row_scale, int rows, int D, int rows_per_b,
-                             const float *mod, int shift_chunk, int scale_chunk,
+int launch_layernorm_mod_fp8(const float *x, uint8_t *q, float *row_scale, int rows, int D, const LnMod &m,
                              const float *g, const float *beta, float eps, cudaStream_t s) {
   if (D % 4 || D > 4 * LN_MAXV * LN_THREADS) return set_error(WAN_EUNSUPPORTED, "layernorm: D=%d", D);
   if (rows == 0) return WAN_OK;
-  layernorm_mod_kernel<uint8_t><<<rows, LN_THREADS, 0, s>>>(x, q, D, rows_per_b, mod, shift_chunk, scale_chunk,
-                                                            g, beta, eps, row_scale);
+  layernorm_mod_kernel<uint8_t><<<rows, LN_THREADS, 0, s>>>(x, q, D, m, g, beta, eps, row_scale);
   WAN_CHECK_LAUNCH("layernorm_mod_fp8");
   return WAN_OK;
 }

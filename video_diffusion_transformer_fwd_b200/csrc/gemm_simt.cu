@@ -94,6 +94,10 @@ __global__ void __launch_bounds__(THREADS) gemm_simt_kernel(const GemmArgs g) {
       for (int j = 0; j < 8; j += 4) {
         float4 xv = g.x_store ? make_float4(0.f, 0.f, 0.f, 0.f) : load4(xr + j);
         float4 gv = gr ? load4(gr + j) : make_float4(1.f, 1.f, 1.f, 1.f);
+        if (gr && g.gate_bias) {
+          const float4 gb = load4(g.gate_bias + nb + j);
+          gv = make_float4(gv.x + gb.x, gv.y + gb.y, gv.z + gb.z, gv.w + gb.w);
+        }
         xv.x = fmaf(gv.x, v[j + 0], xv.x);
         xv.y = fmaf(gv.y, v[j + 1], xv.y);
         xv.z = fmaf(gv.z, v[j + 2], xv.z);

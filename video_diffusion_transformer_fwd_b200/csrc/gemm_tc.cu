@@ -58,6 +58,7 @@ struct TcParams {
   void *C; int ldc;
   float *X; int ldx;
   const float *gate; int gate_stride; int rows_per_gate; int x_store;
+  const float *gate_bias;
   const float *a_scale; const float *b_scale[3];      // FP8: per row of A, per weight segment
   // q/k RMSNorm + RoPE epilogue (EPI_QKNORM)
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
@@ -295,7 +296,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int j16 = 0; j16 < 8; ++j16) {
             float4 gv = make_float4(1.f, 1.f, 1.f, 1.f);
-            if (p.gate) gv = gr ? *reinterpret_cast<const float4 *>(gr + 4 * j16) : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (p.gate) {
+              gv = gr ? *reinterpret_cast<const float4 *>(gr + 4 * j16) : make_float4(0.f, 0.f, 0.f, 0.f);
+              if (p.gate_bias) {
+                const float4 gb = *reinterpret_cast<const float4 *>(p.gate_bias + n + 4 * j16);
+                gv = make_float4(gv.x + gb.x, gv.y + gb.y, gv.z + gb.z, gv.w + gb.w);
+              }
+            }
             const float4 o = make_float4(gv.x * v[4 * j16 + 0], gv.y * v[4 * j16 + 1],
                                          gv.z * v[4 * j16 + 2], gv.w * v[4 * j16 + 3]);
             *reinterpret_cast<float4 *>(buf + lane * 128 + ((j16 ^ (lane & 7)) << 4)) = o;
@@ -423,6 +430,7 @@ bool gemm_tc_supported(const GemmArgs &g) {
   if (g.lda % 8) return false;
   if (g.epi != EPI_RESID && g.ldc % 8) return false;
   if (g.epi == EPI_RESID && (g.ldx % 4 || !aligned16(g.X) || (g.gate && g.gate_stride % 4))) return false;
+  if (g.gate_bias && !aligned16(g.gate_bias)) return false;
   if (g.epi == EPI_QKNORM) {
     for (int i = 0; i < g.nseg; ++i) {
       if (g.ss_col[i] >= 0 && !g.ss) return false;
@@ -460,6 +468,7 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   p.C = g.C; p.ldc = g.ldc; p.X = g.X; p.ldx = g.ldx;
   p.gate = g.gate; p.gate_stride = g.gate_stride; p.rows_per_gate = g.rows_per_gate > 0 ? g.rows_per_gate : 1;
   p.x_store = g.x_store;
+  p.gate_bias = g.gate_bias;
   for (int i = 0; i < 3; ++i) {
     p.gamma[i] = i < g.nseg ? g.gamma[i] : nullptr;
     p.ss_col[i] = i < g.nseg ? g.ss_col[i] : -1;

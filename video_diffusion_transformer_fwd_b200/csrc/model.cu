@@ -64,23 +64,13 @@ __global__ void silu_kernel(const float *__restrict__ x, float *__restrict__ y, 
   if (i < n) y[i] = x[i] / (1.0f + expf(-x[i]));
 }
 
-// hm[b][c][:] = head_mod[c][:] + e[b][:] for the two chunks (shift, scale)
-// of the head, laid out like the blocks' [B, 6, dim] modulation (chunks 0, 1)
-__global__ void head_mod_kernel(const float *__restrict__ head_mod, const float *__restrict__ e,
-                                float *__restrict__ hm, int B, int D) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= B * 2 * D) return;
-  const int d = i % D, c = (i / D) % 2, b = i / (2 * D);
-  hm[((size_t)b * 6 + c) * D + d] = head_mod[c * D + d] + e[(size_t)b * D + d];
-}
-
 int grid_for(size_t n) {
   size_t g = (n + 255) / 256;
   if (g > 148 * 32) g = 148 * 32;
   return g < 1 ? 1 : (int)g;
 }
 
-enum { MW_X, MW_PATCH, MW_CTX, MW_TXT, MW_SIN, MW_H1, MW_E, MW_SE, MW_E0, MW_HMOD, MW_HOUT, MW_BLOCK, MW_COUNT };
+enum { MW_X, MW_PATCH, MW_CTX, MW_TXT, MW_SIN, MW_H1, MW_E, MW_SE, MW_E0, MW_HOUT, MW_BLOCK, MW_COUNT };
 
 struct ModelLayout {
   size_t off[MW_COUNT];
@@ -94,7 +84,7 @@ wan_dims token_dims(const wan_model_dims &m) {
   wan_dims d;
   d.F = m.F; d.H = m.H / 2; d.W = m.W / 2;
   d.dim = m.dim; d.heads = m.heads; d.ffn_dim = m.ffn_dim; d.text_len = m.text_len;
-  d.eps = m.eps; d.dtype = m.dtype;
+  d.eps = m.eps; d.dtype = m.dtype; d.e0_per_token = m.t_per_token;
   return d;
 }
 
@@ -106,6 +96,7 @@ int check_model(const wan_model_dims *m, int B) {
   if (m->text_len > 0 && (m->text_dim < 64 || m->text_dim % 64))
     return set_error(WAN_EINVAL, "text_dim %d must be a positive multiple of 64", m->text_dim);
   if ((m->C_in * 4) % 8) return set_error(WAN_EUNSUPPORTED, "C_in * 4 must be a multiple of 8");
+  if (m->t_per_token != 0 && m->t_per_token != 1) return set_error(WAN_EINVAL, "t_per_token must be 0 or 1");
   const wan_dims d = token_dims(*m);
   if (wan_block_workspace_bytes(&d, B) == 0 && B > 0) return WAN_EINVAL;   // message set by the block check
   return WAN_OK;
@@ -116,6 +107,7 @@ ModelLayout model_layout(const wan_model_dims &m, int B) {
   const size_t es = dtype_size(m.dtype);
   const size_t L = (size_t)m.F * (m.H / 2) * (m.W / 2), BL = (size_t)B * L, D = m.dim;
   const size_t BT = (size_t)B * m.text_len;
+  const size_t NT = m.t_per_token ? BL : (size_t)B;     // timesteps
   const wan_dims d = token_dims(m);
   l.block_bytes = wan_block_workspace_bytes(&d, B);
   const size_t sz[MW_COUNT] = {
@@ -123,12 +115,11 @@ ModelLayout model_layout(const wan_model_dims &m, int B) {
       BL * m.C_in * 4 * es,            // PATCH
       BT * D * es,                     // CTX
       BT * D * es,                     // TXT (text MLP hidden)
-      (size_t)B * m.freq_dim * 4,      // SIN
-      (size_t)B * D * 4,               // H1
-      (size_t)B * D * 4,               // E
-      (size_t)B * D * 4,               // SE
-      (size_t)B * 6 * D * 4,           // E0
-      (size_t)B * 6 * D * 4,           // HMOD
+      NT * m.freq_dim * 4,             // SIN
+      NT * D * 4,                      // H1
+      NT * D * 4,                      // E
+      NT * D * 4,                      // SE
+      NT * 6 * D * 4,                  // E0
       BL * m.C_out * 4 * es,           // HOUT
       l.block_bytes,                   // BLOCK (its ACT buffer also holds the head's LN output)
   };
@@ -200,7 +191,6 @@ int wan_model_forward(const wan_model_dims *dims, int B, const float *latent, co
   float *e = reinterpret_cast<float *>(ws + lay.off[MW_E]);
   float *se = reinterpret_cast<float *>(ws + lay.off[MW_SE]);
   float *e0 = reinterpret_cast<float *>(ws + lay.off[MW_E0]);
-  float *hmod = reinterpret_cast<float *>(ws + lay.off[MW_HMOD]);
   void *hout = ws + lay.off[MW_HOUT];
   char *bws = ws + lay.off[MW_BLOCK];
   const wan_dims tok = token_dims(m);
@@ -223,18 +213,20 @@ int wan_model_forward(const wan_model_dims *dims, int B, const float *latent, co
     g.x_store = 1;
     if ((rc = gemm_any(g, dt, s))) return rc;
   }
-  // time embedding (fp32): e = W2 SiLU(W1 sinusoid(t) + b1) + b2; e0 = Wp SiLU(e) + bp
+  // time embedding (fp32): e = W2 SiLU(W1 sinusoid(t) + b1) + b2; e0 = Wp SiLU(e) + bp,
+  // for B timesteps or, per token, B * L
+  const int NT = m.t_per_token ? BL : B;
   {
     const int half = m.freq_dim / 2;
-    WAN_PROF(WAN_K_MODEL, s, (sinusoid_kernel<<<(B * half + 255) / 256, 256, 0, s>>>(t, sin_, B, m.freq_dim), 0));
+    WAN_PROF(WAN_K_MODEL, s, (sinusoid_kernel<<<(NT * half + 255) / 256, 256, 0, s>>>(t, sin_, NT, m.freq_dim), 0));
     WAN_CHECK_LAUNCH("sinusoid");
     GemmArgs g = {};
-    g.M = B; g.N = D; g.K = m.freq_dim; g.A = sin_; g.lda = m.freq_dim;
+    g.M = NT; g.N = D; g.K = m.freq_dim; g.A = sin_; g.lda = m.freq_dim;
     g.Bseg[0] = w->time_w1; g.bias[0] = w->time_b1; g.segN = D; g.nseg = 1; g.epi = EPI_SILU; g.C = h1; g.ldc = D;
     if ((rc = gemm_any(g, WAN_F32, s))) return rc;
     g.K = D; g.A = h1; g.lda = D; g.Bseg[0] = w->time_w2; g.bias[0] = w->time_b2; g.epi = EPI_STORE; g.C = e;
     if ((rc = gemm_any(g, WAN_F32, s))) return rc;
-    WAN_PROF(WAN_K_MODEL, s, (silu_kernel<<<(B * D + 255) / 256, 256, 0, s>>>(e, se, B * D), 0));
+    WAN_PROF(WAN_K_MODEL, s, (silu_kernel<<<(NT * D + 255) / 256, 256, 0, s>>>(e, se, NT * D), 0));
     WAN_CHECK_LAUNCH("silu");
     g.A = se; g.N = 6 * D; g.segN = 6 * D; g.Bseg[0] = w->proj_w; g.bias[0] = w->proj_b; g.C = e0; g.ldc = 6 * D;
     if ((rc = gemm_any(g, WAN_F32, s))) return rc;
@@ -253,11 +245,10 @@ int wan_model_forward(const wan_model_dims *dims, int B, const float *latent, co
     if ((rc = wan_block_forward(&tok, B, X, T > 0 ? ctx : nullptr, ctx_lens, e0, &blocks[i], rope,
                                 rope_max_pos, bws, lay.block_bytes, stream)))
       return rc;
-  // head: LN(x) (1 + m1) + m0 with m = head_mod + e, then Linear(dim -> C_out * 4)
+  // head: LN(x) (1 + m1) + m0 with (m0, m1) = head_mod + e (read in place), then Linear(dim -> C_out * 4)
   {
-    WAN_PROF(WAN_K_MODEL, s, (head_mod_kernel<<<(B * 2 * D + 255) / 256, 256, 0, s>>>(w->head_mod, e, hmod, B, D), 0));
-    WAN_CHECK_LAUNCH("head_mod");
-    if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(X, act, dt, BL, D, L, hmod, 0, 1, nullptr, nullptr, m.eps, s))))
+    const LnMod hm{e, m.t_per_token ? 1 : L, (size_t)D, 0, 0, w->head_mod, 0, D};
+    if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(X, act, dt, BL, D, hm, nullptr, nullptr, m.eps, s))))
       return rc;
     GemmArgs g = {};
     g.M = BL; g.N = m.C_out * 4; g.K = D; g.A = act; g.lda = D;

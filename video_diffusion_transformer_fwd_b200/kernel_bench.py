@@ -44,6 +44,7 @@ def main():
     ap.add_argument("--blocks", type=int, default=0)
     ap.add_argument("--fp8", action="store_true", help="block: FP8 GEMM mode")
     ap.add_argument("--attn8", action="store_true", help="8-bit attention (block: with FP8 GEMMs)")
+    ap.add_argument("--per-token", action="store_true", help="block: e0 per token [B, L, 6, dim]")
     ap.add_argument("--config", default="a14b-step")
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--L", type=int, default=16384)
@@ -81,12 +82,15 @@ def main():
         dims.dtype = wan.WAN_FP8_ATTN if a.attn8 else wan.WAN_FP8
         w = wan.quantize_block_weights(w)
     acts = synth.block_activations(a.B, cfg.L, cfg.dim, cfg.text_len, cfg.dtype, "cuda", 100)
+    if a.per_token:
+        dims.e0_per_token = 1
+        acts["e0"] = acts["e0"][:, None].expand(a.B, cfg.L, 6, cfg.dim).contiguous()
     rope = wan.rope_freqs(cfg.head_dim, 1024, cfg.theta)
     ws = wan.alloc_workspace(dims, a.B)
     cw = wan.make_weights(w)
     ms, prof = _time(lambda: wan.block_forward(dims, acts["x"], acts["ctx"], acts["e0"], cw, rope, ws),
                      a.iters, a.warmup)
-    print(json.dumps({"what": "block", "config": cfg.name, "B": a.B, "L": cfg.L, "fp8": a.fp8, "attn8": a.attn8, "ms": ms,
+    print(json.dumps({"what": "block", "config": cfg.name, "B": a.B, "L": cfg.L, "fp8": a.fp8, "attn8": a.attn8, "per_token": a.per_token, "ms": ms,
                       "tflops": cfg.block_flops() / ms / 1e9,
                       "gemm_tflops": cfg.gemm_flops() / (prof.get("gemm_tc", 0) or float("nan")) / 1e9,
                       "attn_tflops": cfg.self_attn_flops() / (prof.get("attn_self", 0) or float("nan")) / 1e9,

@@ -37,7 +37,8 @@ class WanError(RuntimeError):
 class wan_dims(ctypes.Structure):
     _fields_ = [("F", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
                 ("dim", ctypes.c_int), ("heads", ctypes.c_int), ("ffn_dim", ctypes.c_int),
-                ("text_len", ctypes.c_int), ("eps", ctypes.c_float), ("dtype", ctypes.c_int)]
+                ("text_len", ctypes.c_int), ("eps", ctypes.c_float), ("dtype", ctypes.c_int),
+                ("e0_per_token", ctypes.c_int)]
 
 
 WEIGHT_FIELDS = ("modulation", "wq", "bq", "wk", "bk", "wv", "bv", "wo", "bo", "gq", "gk",
@@ -56,7 +57,7 @@ class wan_model_dims(ctypes.Structure):
                 ("H", ctypes.c_int), ("W", ctypes.c_int), ("dim", ctypes.c_int),
                 ("heads", ctypes.c_int), ("ffn_dim", ctypes.c_int), ("text_len", ctypes.c_int),
                 ("text_dim", ctypes.c_int), ("freq_dim", ctypes.c_int), ("eps", ctypes.c_float),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("t_per_token", ctypes.c_int)]
 
 
 MODEL_WEIGHT_FIELDS = ("patch_w", "patch_b", "text_w1", "text_b1", "text_w2", "text_b2",
@@ -253,9 +254,9 @@ def dtype_code(t) -> int:
 DTYPE_CODES = {"bf16": WAN_BF16, "f32": WAN_F32, "fp8": WAN_FP8, "fp8attn": WAN_FP8_ATTN}
 
 
-def make_dims(F, H, W, dim, heads, ffn_dim, text_len, eps=1e-6, dtype="bf16") -> wan_dims:
+def make_dims(F, H, W, dim, heads, ffn_dim, text_len, eps=1e-6, dtype="bf16", e0_per_token=False) -> wan_dims:
     code = DTYPE_CODES[dtype] if isinstance(dtype, str) else int(dtype)
-    return wan_dims(F, H, W, dim, heads, ffn_dim, text_len, eps, code)
+    return wan_dims(F, H, W, dim, heads, ffn_dim, text_len, eps, code, 1 if e0_per_token else 0)
 
 
 def dims_of(cfg) -> wan_dims:
@@ -392,10 +393,10 @@ def device_status(stream=None) -> int:
 
 
 def make_model_dims(C_in, C_out, F, H, W, dim, heads, ffn_dim, text_len, text_dim, freq_dim=256,
-                    eps=1e-6, dtype="bf16") -> wan_model_dims:
+                    eps=1e-6, dtype="bf16", t_per_token=False) -> wan_model_dims:
     code = DTYPE_CODES[dtype] if isinstance(dtype, str) else int(dtype)
     return wan_model_dims(C_in, C_out, F, H, W, dim, heads, ffn_dim, text_len, text_dim, freq_dim,
-                          eps, code)
+                          eps, code, 1 if t_per_token else 0)
 
 
 def make_model_weights(w: dict) -> wan_model_weights:
@@ -424,7 +425,7 @@ def alloc_model_workspace(dims: wan_model_dims, B: int, device="cuda"):
 def model_forward(dims: wan_model_dims, latent, t, text, weights, blocks, rope, workspace,
                   ctx_lens=None, out=None, stream=None):
     """Velocity of the whole model: latent [B, C_in, F, H, W] float32, t [B]
-    float32 timesteps (device), text [B, text_len, text_dim] in the compute
+    (or [B, L] with dims.t_per_token) float32 timesteps (device), text [B, text_len, text_dim] in the compute
     dtype. ``blocks`` is a list of block weight dicts or a make_block_array()
     result. Returns out [B, C_out, F, H, W] float32."""
     torch = _torch()
