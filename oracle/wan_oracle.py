@@ -673,3 +673,114 @@ def model_denoise_step(latent, sigma, sigma_next, ctx_cond, ctx_uncond, mw, bloc
     t = np.array([1000.0 * sigma] * 2)
     v = model_forward(lat2, t, ctx, None, mw, blocks, heads, eps, theta, freq_dim)
     return euler_cfg_step(latent, v[0], v[1], guide_scale, sigma, sigma_next)
+
+
+# --------------------------------------------------------------------------
+# UniPC multistep sampler ("Wan2.2 I2V inference trace" (damodev.csdn.net),
+# section 4 "DIT": the latent update "UniPC: x_noise <- step(v, t, x_noise)";
+# "Wan architecture overview", scheduler: Euler or UniPC multistep). The pages
+# name the method only; its steps follow the UniPC paper (Zhao et al., 2023,
+# "UniPC: A Unified Predictor-Corrector Framework for Fast Sampling of
+# Diffusion Models"): the data-prediction form, B(h) = e^h - 1 ("bh2"),
+# predictor UniP-p and corrector UniC-p sharing one model evaluation per step.
+# Readings: flow matching x = (1 - sigma) x0 + sigma eps gives alpha = 1 - sigma
+# and the data prediction x0 = x - sigma v; lambda = log(alpha / sigma);
+# order 2 with one first-order warm-up step and a first-order final step;
+# the schedule's first sigma is below 1 and its last is 0.
+# --------------------------------------------------------------------------
+
+def flow_lambda(sigma: float) -> float:
+    """log(alpha / sigma) with alpha = 1 - sigma (+inf at sigma = 0)."""
+    if sigma == 0.0:
+        return math.inf
+    return math.log(1.0 - sigma) - math.log(sigma)
+
+
+def _unipc_phis(h: float, order: int):
+    """h_phi_1, B(h) and the right-hand side b of the order conditions
+    (data prediction: hh = -h)."""
+    hh = -h
+    h_phi_1 = math.expm1(hh)
+    B_h = math.expm1(hh)
+    h_phi_k = h_phi_1 / hh - 1.0
+    b, fact = [], 1.0
+    for j in range(1, order + 1):
+        b.append(h_phi_k * fact / B_h)
+        fact *= j + 1
+        h_phi_k = h_phi_k / hh - 1.0 / fact
+    return h_phi_1, B_h, np.array(b)
+
+
+def unipc_predict(x, m_hist, sigmas, i: int, order: int):
+    """UniP-p from sigma_i to sigma_{i+1}: m_hist[-1] is m_i (at sigma_i),
+    m_hist[-1-k] the output k steps earlier."""
+    s0, t = sigmas[i], sigmas[i + 1]
+    lam_s0, lam_t = flow_lambda(s0), flow_lambda(t)
+    h = lam_t - lam_s0
+    m0 = np.asarray(m_hist[-1], F64)
+    h_phi_1, B_h, b = _unipc_phis(h, order)
+    x_t = (t / s0) * np.asarray(x, F64) - (1.0 - t) * h_phi_1 * m0
+    if order >= 2:
+        rks = np.array([(flow_lambda(sigmas[i - k]) - lam_s0) / h for k in range(1, order)])
+        D1s = [(np.asarray(m_hist[-1 - k], F64) - m0) / rks[k - 1] for k in range(1, order)]
+        if order == 2:
+            rho = np.array([0.5])
+        else:
+            R = np.stack([np.append(rks, 1.0) ** (j - 1) for j in range(1, order + 1)])
+            rho = np.linalg.solve(R[:-1, :-1], b[:-1])
+        x_t = x_t - (1.0 - t) * B_h * sum(r * d for r, d in zip(rho, D1s))
+    return x_t
+
+
+def unipc_correct(last, m_hist, m_new, sigmas, i: int, order: int):
+    """UniC-p at sigma_i: refines the sample reached from sigma_{i-1} (whose
+    corrected value is ``last``) with the new output m_new at sigma_i;
+    m_hist[-1] is the output at sigma_{i-1}, m_hist[-1-k] k steps earlier."""
+    s0, t = sigmas[i - 1], sigmas[i]
+    lam_s0, lam_t = flow_lambda(s0), flow_lambda(t)
+    h = lam_t - lam_s0
+    m0 = np.asarray(m_hist[-1], F64)
+    h_phi_1, B_h, b = _unipc_phis(h, order)
+    rks = np.array([(flow_lambda(sigmas[i - 1 - k]) - lam_s0) / h for k in range(1, order)] + [1.0])
+    D1s = [(np.asarray(m_hist[-1 - k], F64) - m0) / rks[k - 1] for k in range(1, order)]
+    if order == 1:
+        rho = np.array([0.5])
+    else:
+        R = np.stack([rks ** (j - 1) for j in range(1, order + 1)])
+        rho = np.linalg.solve(R, b)
+    x_t = (t / s0) * np.asarray(last, F64) - (1.0 - t) * h_phi_1 * m0
+    corr = sum(r * d for r, d in zip(rho[:-1], D1s))
+    return x_t - (1.0 - t) * B_h * (corr + rho[-1] * (np.asarray(m_new, F64) - m0))
+
+
+def unipc_sample(x, velocity, sigmas, order: int = 2, corrector: bool = True,
+                 lower_order_final: bool = True):
+    """Run the sampler from sigmas[0] to sigmas[-1] = 0 with one evaluation of
+    ``velocity(x, sigma, i)`` per step (i = 0 .. len(sigmas) - 2). Returns the
+    final sample and the list of samples handed to the evaluations.
+    ``corrector`` False leaves out UniC; ``lower_order_final`` False keeps the
+    full order on the last step."""
+    sigmas = [float(s) for s in sigmas]
+    n = len(sigmas) - 1
+    x = np.asarray(x, F64)
+    m_hist, last, prev_order, seen = [], None, 0, []
+    for i in range(n):
+        seen.append(x)
+        m = x - sigmas[i] * np.asarray(velocity(x, sigmas[i], i), F64)   # data prediction
+        if i > 0 and corrector:
+            x = unipc_correct(last, m_hist, m, sigmas, i, prev_order)
+        m_hist = (m_hist + [m])[-order:]
+        this_order = min(order, n - i if lower_order_final else order, i + 1)   # warm-up, final step
+        last = x
+        x = unipc_predict(x, m_hist, sigmas, i, this_order)
+        prev_order = this_order
+    return x, seen
+
+
+def flow_sigmas(num_steps: int, shift: float = 5.0, sigma_max: float = 0.999) -> np.ndarray:
+    """A flow-matching schedule: num_steps values from sigma_max down to
+    1 / num_steps of it, time-shifted sigma -> s sigma / (1 + (s - 1) sigma),
+    then the final 0."""
+    base = np.linspace(sigma_max, sigma_max / num_steps, num_steps)
+    shifted = shift * base / (1.0 + (shift - 1.0) * base)
+    return np.append(shifted, 0.0)
