@@ -293,6 +293,37 @@ int wan_quantize_fp8(const void *src, int src_dtype, int rows, int cols, int per
 int wan_linear_fp8(int M, int N, int K, const uint8_t *a, const float *a_scale, const uint8_t *w,
                    const float *w_scale, const void *bias, float *out, wan_stream_t stream);
 
+/* UniPC multistep sampler for the latent ("Wan2.2 I2V inference trace",
+ * section 4 "DIT": the latent update "UniPC: x_noise <- step(v, t, x_noise)";
+ * the method of Zhao et al., 2023, "UniPC: A Unified Predictor-Corrector
+ * Framework for Fast Sampling of Diffusion Models", data-prediction form,
+ * B(h) = e^h - 1). With alpha = 1 - sigma, lambda = log(alpha / sigma) and
+ * the data prediction m_i = x_i - sigma_i v_i of evaluation i, one step
+ * corrects the sample reached by step i - 1 with m_i (UniC) and predicts the
+ * sample at sigma_{i+1} (UniP); orders 1 and 2, the first step first order.
+ *
+ * wan_unipc_coefficients (host only) -- the step's eight coefficients
+ *   x_c    = c[0] x + c[1] last + c[2] m_{i-1} + c[3] m_{i-2} + c[4] m_i
+ *   x_next = c[5] x_c + c[6] m_i + c[7] m_{i-1}
+ *   sigmas  host double [num_sigmas], decreasing in [0, 1), only the last 0;
+ *           num_sigmas - 1 model evaluations, step in [0, num_sigmas - 2].
+ *   order   1 or 2; lower_order_final: the last step first order (a last
+ *           step onto sigma = 0 is always first order).
+ * wan_unipc_step -- applies one step in place, n float32 elements:
+ *   v = v_uncond + guide_scale (v_cond - v_uncond) (v_uncond NULL: v_cond),
+ *   m_out = x - sigma_i v, last = x_c, x = x_next (coef from the call above
+ *   with the same step). m_prev1 / m_prev2 are m_{i-1} / m_{i-2} (may be
+ *   NULL where their coefficients are 0); last is read only when c[1] != 0.
+ *   m_out, m_prev1, m_prev2 must be distinct buffers (the caller rotates 3).
+ * Errors: WAN_EINVAL (schedule, step, NULL), WAN_EUNSUPPORTED (order > 2,
+ *         dtype), WAN_EALIGN. */
+int wan_unipc_coefficients(const double *sigmas, int num_sigmas, int step, int order,
+                           int lower_order_final, double coef[8]);
+int wan_unipc_step(float *x, float *last, float *m_out, const float *m_prev1,
+                   const float *m_prev2, const void *v_cond, const void *v_uncond, int v_dtype,
+                   size_t n, float guide_scale, float sigma, const double coef[8],
+                   wan_stream_t stream);
+
 /* wan_attention_8bit -- 8-bit flash attention ([DIGEST] inference-optimisation
  * table, "8-bit FlashAttention": int8 for S = Q K^T, FP8 for O = P V, fp32
  * accumulation across key blocks), non-causal, head_dim 128.

@@ -96,9 +96,19 @@ class ModelDenoiseStep:
             return "high"
         return "low"
 
-    def step(self, sigma: float, sigma_next: float, guide_scale: float, stream=None):
+    def _guide(self, name, guide_scale):
+        """A (low-noise, high-noise) pair picks the expert's scale ([WALK]
+        sampling-loop snippet: e.g. (3.0, 4.0) for text-to-video)."""
+        if isinstance(guide_scale, (tuple, list)):
+            return guide_scale[1] if name == "high" else guide_scale[0]
+        return guide_scale
+
+    def velocity(self, sigma: float, stream=None):
+        """The model on the CFG pair at t = 1000 sigma: self.v[0] (cond),
+        self.v[1] (uncond). Returns the expert used."""
         s = wan._stream(stream)
-        mw, blocks = self.experts[self.expert(sigma)]
+        name = self.expert(sigma)
+        mw, blocks = self.experts[name]
         self.lat2[0].copy_(self.latent)
         self.lat2[1].copy_(self.latent)
         self.t.fill_(1000.0 * sigma)
@@ -106,7 +116,20 @@ class ModelDenoiseStep:
                                         wan._ptr(self.text), wan._ptr(self.ctx_lens), mw, blocks,
                                         len(blocks), self.rope.data_ptr(), self.rope.shape[0],
                                         self.v.data_ptr(), self.ws.data_ptr(), self.ws.numel(), s))
+        return name
+
+    def step(self, sigma: float, sigma_next: float, guide_scale, stream=None):
+        """Euler step from sigma to sigma_next."""
+        name = self.velocity(sigma, stream)
         wan.check(wan.wan_euler_cfg_step(self.latent.data_ptr(), self.v[0].data_ptr(),
                                          self.v[1].data_ptr(), wan.WAN_F32, self.latent.numel(),
-                                         guide_scale, sigma, sigma_next, s))
+                                         self._guide(name, guide_scale), sigma, sigma_next,
+                                         wan._stream(stream)))
+        return self.latent
+
+    def unipc_step(self, sampler: "wan.UniPCSampler", guide_scale, stream=None):
+        """One UniPC step (the sampler's x is this latent): the model at the
+        sampler's current sigma, then the fused UniPC update."""
+        name = self.velocity(sampler.sigma, stream)
+        sampler.step(self.v[0], self.v[1], self._guide(name, guide_scale), stream)
         return self.latent

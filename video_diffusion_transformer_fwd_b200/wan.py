@@ -92,6 +92,10 @@ _SIGS = {
     "wan_quantize_fp8": (_c_int, [_vp, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp]),
     "wan_linear_fp8": (_c_int, [_c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "wan_attention_8bit_workspace_bytes": (_sz, [_c_int, _c_int, _c_int, _c_int]),
+    "wan_unipc_coefficients": (_c_int, [ctypes.POINTER(ctypes.c_double), _c_int, _c_int, _c_int, _c_int,
+                                        ctypes.POINTER(ctypes.c_double)]),
+    "wan_unipc_step": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _sz, ctypes.c_float, ctypes.c_float,
+                                ctypes.POINTER(ctypes.c_double), _vp]),
     "wan_attention_8bit": (_c_int, [_c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
                                     _vp, _sz, _vp]),
     "wan_model_forward": (_c_int, [ctypes.POINTER(wan_model_dims), _c_int, _vp, _vp, _vp, _vp,
@@ -196,6 +200,16 @@ def wan_attention_8bit_workspace_bytes(B, heads, Lq, Lk):
 def wan_attention_8bit(B, heads, Lq, Lk, q, k, v, o, k_lens, scale, workspace, ws_bytes, stream):
     return load().wan_attention_8bit(B, heads, Lq, Lk, q, k, v, o, k_lens, scale, workspace, ws_bytes,
                                      stream)
+
+
+def wan_unipc_coefficients(sigmas, num_sigmas, step, order, lower_order_final, coef):
+    return load().wan_unipc_coefficients(sigmas, num_sigmas, step, order, lower_order_final, coef)
+
+
+def wan_unipc_step(x, last, m_out, m_prev1, m_prev2, v_cond, v_uncond, v_dtype, n, guide_scale, sigma, coef,
+                   stream):
+    return load().wan_unipc_step(x, last, m_out, m_prev1, m_prev2, v_cond, v_uncond, v_dtype, n, guide_scale,
+                                 sigma, coef, stream)
 
 
 def wan_device_status(stream):
@@ -440,3 +454,44 @@ def model_forward(dims: wan_model_dims, latent, t, text, weights, blocks, rope, 
                             out.data_ptr(), workspace.data_ptr(),
                             workspace.numel() * workspace.element_size(), _stream(stream)))
     return out
+
+
+class UniPCSampler:
+    """State of the UniPC sampler over one latent (see wan_unipc_step): the
+    schedule, the step index, the corrected previous sample and a ring of
+    three data predictions. ``x`` (float32, device) is updated in place."""
+
+    def __init__(self, x, sigmas, order=2, lower_order_final=True):
+        torch = _torch()
+        self.x = x
+        self.sigmas = [float(s) for s in sigmas]
+        self.n = len(self.sigmas) - 1
+        self.order, self.lof = order, lower_order_final
+        self.i = 0
+        self.last = torch.empty_like(x)
+        self.ring = [torch.empty_like(x) for _ in range(3)]
+        self._sig = (ctypes.c_double * len(self.sigmas))(*self.sigmas)
+        self._coef = (ctypes.c_double * 8)()
+
+    @property
+    def sigma(self) -> float:
+        return self.sigmas[self.i]
+
+    def coefficients(self, step=None):
+        check(wan_unipc_coefficients(self._sig, len(self.sigmas), self.i if step is None else step, self.order,
+                                     1 if self.lof else 0, self._coef))
+        return list(self._coef)
+
+    def step(self, v_cond, v_uncond=None, guide_scale=1.0, stream=None):
+        if self.i >= self.n:
+            raise RuntimeError("UniPC schedule finished")
+        self.coefficients()
+        i = self.i
+        m_out = self.ring[i % 3]
+        m1 = self.ring[(i - 1) % 3] if i >= 1 else None
+        m2 = self.ring[(i - 2) % 3] if i >= 2 else None
+        check(wan_unipc_step(self.x.data_ptr(), self.last.data_ptr(), m_out.data_ptr(), _ptr(m1), _ptr(m2),
+                             v_cond.data_ptr(), _ptr(v_uncond), dtype_code(v_cond), self.x.numel(), guide_scale,
+                             self.sigmas[i], self._coef, _stream(stream)))
+        self.i += 1
+        return self.x
