@@ -5,16 +5,19 @@
 //
 // One CTA = 2 query tiles of 128 rows of one (sequence, head):
 //   warps 0..3 / 4..7  softmax of query tile 0 / 1: thread = one query row;
-//               reads its row of S (128 keys, fp32) from TMEM, keeps a running
-//               max m (log2 domain) and sum l, writes P = exp2(S c - m) as bf16
-//               back into the first 64 columns of the same TMEM region, and
+//               loads its row of S (128 keys, fp32) from TMEM and releases
+//               the S columns at once, keeps a running max m (log2 domain)
+//               and sum l, and writes P = exp2(S c - m) as bf16 into a
+//               shared-memory tile in the MMA's swizzled K-major layout; it
 //               rescales its O row in TMEM only when m grows by more than 8
 //               (P stays <= 2^8 otherwise, the final O / l is unchanged);
-//   warp 8      MMA issuer: S_i = Q_i K_j^T (A, B from shared memory), then
-//               O_i += P_i V_j (A = P from TMEM, B = V, MN-major, from
-//               shared memory);
-//   warp 9      TMA producer: Q tiles once, then K_j and V_j alternately into
-//               a 4-slot ring of 32 KB slots (128-byte swizzle).
+//   warp 8      MMA issuer: S_i(j+1) = Q_i K_{j+1}^T as soon as both the K
+//               tile and the S_i columns are free (while the softmax of tile
+//               j still runs), then O_i += P_i(j) V_j (A = P, B = V MN-major,
+//               both from shared memory);
+//   warp 9      TMA producer: Q tiles once, then K tiles into a 2-slot ring
+//               (K_{j+2} as soon as S(j) is done) and V tiles into one slot
+//               (V_{j+1} once PV(j) is done), 32 KB each (128-byte swizzle).
 // TMEM: S_0 | S_1 | O_0 | O_1, 128 fp32 columns each (512 total).
 // Every wait is bounded (sm100::mbar_wait); keys at or beyond the sequence's
 // key length are masked; rows of a tile beyond Lq are computed but not stored.
@@ -29,15 +32,15 @@ using namespace sm100;
 constexpr int D = 128;                 // head_dim
 constexpr int TQ = 128;                // query rows per tile
 constexpr int TK = 128;                // keys per tile
-constexpr int NSLOT = 4;               // K/V ring slots
-constexpr int TILE_BYTES = 128 * D * 2;  // 32 KB: one Q, K or V tile (two 64-column boxes)
+constexpr int NSLOT = 3;               // K slots 0, 1 and the V slot
+constexpr int TILE_BYTES = 128 * D * 2;  // 32 KB: one Q, K, V or P tile (two 64-column boxes)
 constexpr int BOX_BYTES = TILE_BYTES / 2;
 constexpr int THREADS = 320;                // 8 softmax warps + MMA warp + TMA warp
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC_S = idesc_bf16(TQ, TK, 0);
 constexpr uint32_t IDESC_O = idesc_bf16(TQ, D, 1);
 constexpr float RESCALE_THRESHOLD = 8.0f;   // log2 units
-constexpr int SMEM_BYTES = 1024 + 2 * TILE_BYTES + NSLOT * TILE_BYTES + 256;
+constexpr int SMEM_BYTES = 1024 + 4 * TILE_BYTES + NSLOT * TILE_BYTES + 256;   // Q_0, Q_1, P_0, P_1, ring
 
 struct FaParams {
   int B, heads, Lq, Lk;
@@ -83,20 +86,26 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = smem;                               // 2 tiles
-  uint8_t *sKV = smem + 2 * TILE_BYTES;             // NSLOT tiles
+  uint8_t *sP = smem + 2 * TILE_BYTES;              // 2 tiles
+  uint8_t *sKV = smem + 4 * TILE_BYTES;             // NSLOT tiles
   uint64_t *bars = reinterpret_cast<uint64_t *>(sKV + NSLOT * TILE_BYTES);
   uint64_t *q_full = bars;
-  uint64_t *kv_full = bars + 1;
+  uint64_t *kv_full = bars + 1;                     // [0], [1]: K slots; [2]: V slot
   uint64_t *kv_empty = bars + 1 + NSLOT;
-  uint64_t *s_full = bars + 1 + 2 * NSLOT;
-  uint64_t *p_ready = s_full + 2;
-  uint64_t *pv_done = p_ready + 2;
+  uint64_t *s_full = bars + 1 + 2 * NSLOT;          // S_i computed
+  uint64_t *s_free = s_full + 2;                    // S_i read by its softmax
+  uint64_t *p_full = s_free + 2;                    // P_i written to shared memory
+  uint64_t *pv_done = p_full + 2;                   // O_i += P_i V done (P_i free, O_i stable)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(pv_done + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -121,7 +130,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&p_ready[i]), 4);
+      mbar_init(smem_u32(&s_free[i]), 4);
+      mbar_init(smem_u32(&p_full[i]), 4);
       mbar_init(smem_u32(&pv_done[i]), 1);
     }
     *abort_flag = 0;
@@ -135,6 +145,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // K_j sits in slot j % 2 (its (j / 2)-th fill); V_j in slot 2 (its j-th fill)
+  auto kslot = [](int j) { return j & 1; };
+  auto kphase = [](int j) { return (uint32_t)((j >> 1) & 1); };
+  constexpr int VSLOT = 2;
 
   if (warp >= 8) {
     if (warp == 9) {
@@ -149,22 +163,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int half = 0; half < 2; ++half)
             tma_load_3d(smem_u32(sQ + i * TILE_BYTES + half * BOX_BYTES), &tmQ, h * D + half * 64,
                         q0 + i * TQ, b, qb);
-        int slot = 0;
-        uint32_t phase = 0;
-        int fills[NSLOT] = {0, 0, 0, 0};
-        bool ok = true;
+        int fills[NSLOT] = {0, 0, 0};
+        auto load = [&](int slot, uint32_t empty_phase, const CUtensorMap *tm, int j) {
+          if (!mbar_wait(smem_u32(&kv_empty[slot]), empty_phase, abort_flag, p.watchdog, 0x201)) return false;
+          const uint32_t fb = smem_u32(&kv_full[slot]);
+          mbar_arrive_expect_tx(fb, TILE_BYTES);
+          for (int half = 0; half < 2; ++half)
+            tma_load_3d(smem_u32(sKV + slot * TILE_BYTES + half * BOX_BYTES), tm, h * D + half * 64, j * TK, b, fb);
+          ++fills[slot];
+          return true;
+        };
+        // K_0, K_1, V_0, then K_{j+2} (frees after S(j)) before V_{j+1} (frees after PV(j))
+        bool ok = load(kslot(0), kphase(0) ^ 1, &tmK, 0);
+        if (ok && nkt > 1) ok = load(kslot(1), kphase(1) ^ 1, &tmK, 1);
+        if (ok) ok = load(VSLOT, 1, &tmV, 0);
         for (int j = 0; j < nkt && ok; ++j) {
-          for (int kv = 0; kv < 2; ++kv) {
-            if (!mbar_wait(smem_u32(&kv_empty[slot]), phase ^ 1, abort_flag, p.watchdog, 0x201)) { ok = false; break; }
-            const uint32_t fb = smem_u32(&kv_full[slot]);
-            mbar_arrive_expect_tx(fb, TILE_BYTES);
-            const CUtensorMap *tm = kv == 0 ? &tmK : &tmV;
-            for (int half = 0; half < 2; ++half)
-              tma_load_3d(smem_u32(sKV + slot * TILE_BYTES + half * BOX_BYTES), tm, h * D + half * 64,
-                          j * TK, b, fb);
-            ++fills[slot];
-            if (++slot == NSLOT) { slot = 0; phase ^= 1; }
-          }
+          if (j + 2 < nkt) ok = load(kslot(j + 2), kphase(j + 2) ^ 1, &tmK, j + 2);
+          if (ok && j + 1 < nkt) ok = load(VSLOT, ((j + 1) & 1) ^ 1, &tmV, j + 1);
         }
         int never = 0;
         mbar_wait(qb, 0, &never, p.watchdog, 0x202);
@@ -174,17 +189,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     } else if (warp == 8) {
       // ------------------------------------------------ MMA issuer
       if (lane == 0 && nkt > 0) {
-        // Issue order per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1). A
-        // tile's next S reuses the TMEM columns its P occupies; tcgen05.mma ops
-        // of one CTA execute in issue order, so S_i(j+1) is issued right behind
-        // PV_i(j) and each query tile only waits for its own softmax.
+        // Per key tile j: S_0(j+1), S_1(j+1) as soon as K_{j+1} has landed
+        // and each S_i(j) has been read; then PV_0(j), PV_1(j) once V_j has
+        // landed and each P_i(j) is written. The tensor pipe computes the next
+        // scores while the softmax still works on the current ones.
         bool ok = mbar_wait(smem_u32(q_full), 0, abort_flag, p.watchdog, 0x211);
-        int slot = 0;
-        uint32_t phase = 0;
-        auto next = [&]() { if (++slot == NSLOT) { slot = 0; phase ^= 1; } };
         auto issue_s = [&](int i, uint32_t kbase) {
           const uint32_t qbase = smem_u32(sQ + i * TILE_BYTES);
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
             mma_ss(tmem + i * TK, desc_kmajor_sw128(qbase + off), desc_kmajor_sw128(kbase + off), IDESC_S, kk > 0);
@@ -192,50 +204,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           tc_commit(smem_u32(&s_full[i]));
         };
         auto issue_pv = [&](int i, uint32_t vbase, int j) {
-  #pragma unroll
-          for (int kk = 0; kk < TK / 16; ++kk)
-            mma_ts(tmem + 2 * TK + i * D, tmem + i * TK + kk * 8,
+          const uint32_t pbase = smem_u32(sP + i * TILE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < TK / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
+            mma_ss(tmem + 2 * TK + i * D, desc_kmajor_sw128(pbase + off),
                    desc_mnmajor_sw128(vbase + kk * 16 * 128, BOX_BYTES, 1024), IDESC_O, (j > 0 || kk > 0));
+          }
           tc_commit(smem_u32(&pv_done[i]));
         };
         // prologue: S_0(0), S_1(0)
-        int kslot = slot;
-        if (ok && mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x212)) {
+        if (ok && mbar_wait(smem_u32(&kv_full[kslot(0)]), kphase(0), abort_flag, p.watchdog, 0x212)) {
           tc_fence_after();
-          const uint32_t kbase = smem_u32(sKV + slot * TILE_BYTES);
+          const uint32_t kbase = smem_u32(sKV + kslot(0) * TILE_BYTES);
           issue_s(0, kbase);
           issue_s(1, kbase);
-          tc_commit(smem_u32(&kv_empty[kslot]));
-          next();
+          tc_commit(smem_u32(&kv_empty[kslot(0)]));
         } else {
           ok = false;
         }
         for (int j = 0; j < nkt && ok; ++j) {
-          if (!mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x214)) break;   // V_j
-          const int vslot = slot;
-          const uint32_t vbase = smem_u32(sKV + slot * TILE_BYTES);
-          next();
-          const bool more = j + 1 < nkt;
-          uint32_t kbase = 0;
-          kslot = slot;
-          if (!mbar_wait(smem_u32(&p_ready[0]), j & 1, abort_flag, p.watchdog, 0x215)) break;
+          if (j + 1 < nkt) {
+            const int ks = kslot(j + 1);
+            if (!mbar_wait(smem_u32(&kv_full[ks]), kphase(j + 1), abort_flag, p.watchdog, 0x213)) break;
+            const uint32_t kbase = smem_u32(sKV + ks * TILE_BYTES);
+            if (!mbar_wait(smem_u32(&s_free[0]), j & 1, abort_flag, p.watchdog, 0x214)) break;
+            tc_fence_after();
+            issue_s(0, kbase);
+            if (!mbar_wait(smem_u32(&s_free[1]), j & 1, abort_flag, p.watchdog, 0x215)) break;
+            tc_fence_after();
+            issue_s(1, kbase);
+            tc_commit(smem_u32(&kv_empty[ks]));
+          }
+          if (!mbar_wait(smem_u32(&kv_full[VSLOT]), j & 1, abort_flag, p.watchdog, 0x216)) break;
+          const uint32_t vbase = smem_u32(sKV + VSLOT * TILE_BYTES);
+          if (!mbar_wait(smem_u32(&p_full[0]), j & 1, abort_flag, p.watchdog, 0x217)) break;
           tc_fence_after();
           issue_pv(0, vbase, j);
-          if (more) {
-            if (!mbar_wait(smem_u32(&kv_full[slot]), phase, abort_flag, p.watchdog, 0x216)) break;   // K_{j+1}
-            tc_fence_after();
-            kbase = smem_u32(sKV + slot * TILE_BYTES);
-            next();
-            issue_s(0, kbase);
-          }
-          if (!mbar_wait(smem_u32(&p_ready[1]), j & 1, abort_flag, p.watchdog, 0x217)) break;
+          if (!mbar_wait(smem_u32(&p_full[1]), j & 1, abort_flag, p.watchdog, 0x218)) break;
           tc_fence_after();
           issue_pv(1, vbase, j);
-          tc_commit(smem_u32(&kv_empty[vslot]));
-          if (more) {
-            issue_s(1, kbase);
-            tc_commit(smem_u32(&kv_empty[kslot]));
-          }
+          tc_commit(smem_u32(&kv_empty[VSLOT]));
         }
       }
     }
@@ -243,10 +252,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ------------------------------------------------ softmax (warps 0..7)
     const int i = warp >> 2;                       // query tile
     const int qw = warp & 3;                       // TMEM lane quarter
-    const int row = q0 + i * TQ + qw * 32 + lane;  // query row in the sequence
+    const int r = qw * 32 + lane;                  // row in the tile
+    const int row = q0 + i * TQ + r;               // query row in the sequence
     const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + i * TK;
     const uint32_t o_addr = tmem + lane_off + 2 * TK + i * D;
+    // this row of P_i in the 128-byte swizzled K-major layout: box (64 keys),
+    // row r at r * 128 bytes, 16-byte chunk c at (c ^ (r & 7)) * 16
+    const uint32_t p_row = smem_u32(sP + i * TILE_BYTES) + r * 128;
     float m = -INFINITY, l = 0.f;
     // logit scale of this row: scale * log2(e), times q's RMS factor when the
     // QKV epilogue left q un-normalised (q_ss holds the row's sum of squares)
@@ -265,6 +278,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[c * 32]));
       tmem_ld_wait();
+      // S_i is in registers: its TMEM columns may take S_i(j+1)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&s_free[i]));
       const int kvalid = kl - j * TK;              // keys of this tile that are valid
       const bool full_tile = kvalid >= TK;         // uniform across the CTA
       if (!full_tile) {
@@ -288,32 +305,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const float mnew = need ? tmax : m;
       const float alpha = (need && j > 0) ? ex2(m - mnew) : 1.0f;
       m = mnew;
-      // P = exp2(s c - m) as bf16 pairs into the first 64 columns of S_i
-      // (ex2.approx on the MUFU unit; measured, it is not the limiter here).
+      // P = exp2(s c - m) as bf16 pairs, packed into s[0..63]
       const float2 c2 = make_float2(crow, crow);
       const float2 nm2 = make_float2(-m, -m);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 x = ffma2(make_float2(__uint_as_float(s[c * 32 + 2 * e]), __uint_as_float(s[c * 32 + 2 * e + 1])), c2, nm2);
-          const float2 pp = make_float2(ex2(x.x), ex2(x.y));
-          if (e & 1) acc1 = fadd2(acc1, pp); else acc0 = fadd2(acc0, pp);
-          pk[e] = pack_bf16(pp.x, pp.y);
-        }
-        tmem_st16(s_addr + c * 16, pk);
+      for (int e = 0; e < 64; ++e) {
+        const float2 x = ffma2(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), c2, nm2);
+        const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+        if (e & 1) acc1 = fadd2(acc1, pp); else acc0 = fadd2(acc0, pp);
+        s[e] = pack_bf16(pp.x, pp.y);
       }
       const float2 acc = fadd2(acc0, acc1);
       l = l * alpha + (acc.x + acc.y);
-      // O rescale after P is out of registers (the PV MMA of this tile is
-      // only issued after p_ready); TMEM accesses are warp-collective, so a
-      // warp rescales when any of its rows must
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
+      // P_i and O_i are still in use by PV_i(j-1) until it completes
+      if (j > 0) {
         if (!mbar_wait(smem_u32(&pv_done[i]), (j - 1) & 1, abort_flag, p.watchdog, 0x222)) ok = false;
-        __syncwarp();
         tc_fence_after();
+      }
+      // O rescale (TMEM accesses are warp-collective: a warp rescales when
+      // any of its rows must)
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           uint32_t o[16];
@@ -323,11 +335,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           tmem_st16(o_addr + c * 16, o);
         }
+        tmem_st_wait();
       }
-      tmem_st_wait();
+      // P row -> shared memory: keys 8c .. 8c + 7 form 16-byte chunk c
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint32_t addr = p_row + (c >> 3) * BOX_BYTES + ((((uint32_t)c & 7u) ^ ((uint32_t)r & 7u)) << 4);
+        st_shared_v4(addr, s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&p_ready[i]));
+      if (lane == 0) mbar_arrive(smem_u32(&p_full[i]));
       if (!ok) break;
     }
     // epilogue: O / l -> bf16
