@@ -403,10 +403,12 @@ attn8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 #pragma unroll
       for (int a = 0; a < 8; ++a) mx[a] = fmax3(__uint_as_float(s[a]), __uint_as_float(s[8 + a]), __uint_as_float(s[16 + a]));
 #pragma unroll
-      for (int k = 24; k < 128; k += 16) {
+      for (int k = 24; k < 120; k += 16) {
 #pragma unroll
         for (int a = 0; a < 8; ++a) mx[a] = fmax3(mx[a], __uint_as_float(s[k + a]), __uint_as_float(s[k + 8 + a]));
       }
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx[a] = fmaxf(mx[a], __uint_as_float(s[120 + a]));
       const float traw = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
       const float tmax = (traw - MAGIC_F) * crow;
       const bool need = (tmax > m) || (m == -INFINITY);

@@ -292,9 +292,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // row max of the raw scores (the scale c is positive), 3-input max tree
       float mx[8];
 #pragma unroll
-      for (int a = 0; a < 8; ++a) mx[a] = fmax3(__uint_as_float(s[a]), __uint_as_float(s[8 + a]), __uint_as_float(s[16 + a]));
+      for (int a = 0; a < 8; ++a) mx[a] = fmaxf(__uint_as_float(s[a]), __uint_as_float(s[8 + a]));
 #pragma unroll
-      for (int k = 24; k < 128; k += 16) {
+      for (int k = 16; k < 128; k += 16) {
 #pragma unroll
         for (int a = 0; a < 8; ++a) mx[a] = fmax3(mx[a], __uint_as_float(s[k + a]), __uint_as_float(s[k + 8 + a]));
       }
@@ -308,15 +308,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // P = exp2(s c - m) as bf16 pairs, packed into s[0..63]
       const float2 c2 = make_float2(crow, crow);
       const float2 nm2 = make_float2(-m, -m);
-      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+      float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
       for (int e = 0; e < 64; ++e) {
         const float2 x = ffma2(make_float2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), c2, nm2);
         const float2 pp = make_float2(ex2(x.x), ex2(x.y));
-        if (e & 1) acc1 = fadd2(acc1, pp); else acc0 = fadd2(acc0, pp);
+        acc = fadd2(acc, pp);
         s[e] = pack_bf16(pp.x, pp.y);
       }
-      const float2 acc = fadd2(acc0, acc1);
       l = l * alpha + (acc.x + acc.y);
       // P_i and O_i are still in use by PV_i(j-1) until it completes
       if (j > 0) {
