@@ -13,6 +13,8 @@
 
 namespace wan {
 
+int sm_count();   // SMs of the current device (tma_host.cu)
+
 // ----------------------------------------------------------------------------
 // m[b][c][:] = modulation[c][:] + e0[b][c][:]   (e = (modulation + e0).chunk(6))
 // ----------------------------------------------------------------------------
@@ -203,99 +205,163 @@ int launch_quant_tensor(const void *src, int dtype, size_t n, uint8_t *q, float 
 // ----------------------------------------------------------------------------
 // LayerNorm over D (population variance, eps inside the square root), then
 // either the AdaLN modulation (1 + scale) * u + shift with chunks taken from
-// m[b] (norm1 / norm2), or an affine g * u + beta (norm3). One CTA per row;
-// the row stays in registers between the two passes (exact two-pass stats).
+// m[b] (norm1 / norm2), or an affine g * u + beta (norm3). A CTA of 256
+// threads normalises one row at a time with the row in registers (exact
+// two-pass statistics: the mean, then the sum of squared deviations), and
+// walks rows blockIdx.x, blockIdx.x + gridDim.x, ... (two CTAs per SM): the
+// next row's loads are issued before the current row is reduced and stored,
+// so HBM reads stay in flight through the reductions. Each block reduction
+// takes one barrier (partials double-buffered by reduction parity).
 // ----------------------------------------------------------------------------
 constexpr int LN_THREADS = 256;
 constexpr int LN_MAXV = 8;          // float4 per thread: D <= 8192
+constexpr int LN_CTAS_PER_SM = 2;   // two rows in flight per CTA (the next one prefetched)
+
+// Sum (MAX = false) or maximum over the CTA; `red` is this reduction's slot of
+// 32 floats, alternating between two slots from one reduction to the next.
+template <bool MAX>
+__device__ __forceinline__ float block_reduce_1sync(float v, float *red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  constexpr int NW = LN_THREADS / 32;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = MAX ? fmaxf(v, w) : v + w;
+  }
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float t = (lane < NW) ? red[lane] : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float w = __shfl_xor_sync(0xffffffffu, t, o);
+    t = MAX ? fmaxf(t, w) : t + w;
+  }
+  return t;
+}
+
+template <int VPT>
+__device__ __forceinline__ void ln_load_row(float4 (&v)[VPT], const float *__restrict__ xr, int nv) {
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int c = threadIdx.x + i * LN_THREADS;
+    if (c < nv) v[i] = load4(xr + 4 * c);
+  }
+}
 
 // With OutT = uint8_t the modulated row is quantized to e4m3 with its own
-// scale (written to row_scale), the input of an FP8 GEMM.
-template <typename OutT>
-__global__ void __launch_bounds__(LN_THREADS)
-layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int D, const LnMod md,
+// scale (written to row_scale), the input of an FP8 GEMM. VPT = float4
+// chunks per thread (ceil(D / 1024)).
+template <typename OutT, int VPT>
+__global__ void __launch_bounds__(LN_THREADS, LN_CTAS_PER_SM)
+layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int rows, int D, const LnMod md,
                      const float *__restrict__ g, const float *__restrict__ beta, float eps,
                      float *__restrict__ row_scale) {
-  __shared__ float red[32];
-  const int row = blockIdx.x;
-  const float *xr = x + (size_t)row * D;
+  __shared__ float red[2][32];
   const int nv = D >> 2;
-  float4 v[LN_MAXV];
-  float s = 0.f;
+  int row = blockIdx.x;
+  if (row >= rows) return;
+  int k = 0;                               // reductions so far (selects the partials slot)
+  float4 v[VPT], nxt[VPT];
+  ln_load_row<VPT>(v, x + (size_t)row * D, nv);
+  for (; row < rows; row += gridDim.x) {
+    const int nrow = row + gridDim.x;      // uniform across the CTA
+    if (nrow < rows) ln_load_row<VPT>(nxt, x + (size_t)nrow * D, nv);
+    float s = 0.f;
 #pragma unroll
-  for (int i = 0; i < LN_MAXV; ++i) {
-    const int c = threadIdx.x + i * LN_THREADS;
-    if (c < nv) {
-      v[i] = load4(xr + 4 * c);
-      s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
-    }
-  }
-  const float mean = block_sum(s, red) / (float)D;
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < LN_MAXV; ++i) {
-    const int c = threadIdx.x + i * LN_THREADS;
-    if (c < nv) {
-      const float a = v[i].x - mean, b = v[i].y - mean, cc = v[i].z - mean, d = v[i].w - mean;
-      ss += (a * a + b * b) + (cc * cc + d * d);
-    }
-  }
-  const float var = block_sum(ss, red) / (float)D;
-  const float rstd = 1.0f / sqrtf(var + eps);
-  const float *mshift = nullptr, *mscale = nullptr, *bshift = nullptr, *bscale = nullptr;
-  if (md.mod) {
-    const float *mrow = md.mod + (size_t)(row / md.rows_div) * md.row_stride;
-    mshift = mrow + md.shift_off;
-    mscale = mrow + md.scale_off;
-    if (md.bias) {
-      bshift = md.bias + md.bias_shift_off;
-      bscale = md.bias + md.bias_scale_off;
-    }
-  }
-  OutT *orow = out + (size_t)row * D;
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < LN_MAXV; ++i) {
-    const int c = threadIdx.x + i * LN_THREADS;
-    if (c < nv) {
-      float4 u = make_float4((v[i].x - mean) * rstd, (v[i].y - mean) * rstd,
-                             (v[i].z - mean) * rstd, (v[i].w - mean) * rstd);
-      float4 a, b;
-      if (md.mod) {
-        float4 sc = load4(mscale + 4 * c), sh = load4(mshift + 4 * c);
-        if (bshift) {
-          const float4 bs = load4(bscale + 4 * c), bh = load4(bshift + 4 * c);
-          sc = make_float4(sc.x + bs.x, sc.y + bs.y, sc.z + bs.z, sc.w + bs.w);
-          sh = make_float4(sh.x + bh.x, sh.y + bh.y, sh.z + bh.z, sh.w + bh.w);
-        }
-        a = make_float4(1.f + sc.x, 1.f + sc.y, 1.f + sc.z, 1.f + sc.w);
-        b = sh;
-      } else {
-        a = load4(g + 4 * c);
-        b = load4(beta + 4 * c);
-      }
-      u.x = fmaf(u.x, a.x, b.x);
-      u.y = fmaf(u.y, a.y, b.y);
-      u.z = fmaf(u.z, a.z, b.z);
-      u.w = fmaf(u.w, a.w, b.w);
-      if constexpr (sizeof(OutT) == 1) {
-        v[i] = u;
-        amax = fmaxf(amax, absmax4(u));
-      } else {
-        store4(orow + 4 * c, u);
-      }
-    }
-  }
-  if constexpr (sizeof(OutT) == 1) {
-    amax = block_max(amax, red);
-    const float inv = e4m3_inv_scale(amax);
-    uint32_t *qr = reinterpret_cast<uint32_t *>(orow);
-#pragma unroll
-    for (int i = 0; i < LN_MAXV; ++i) {
+    for (int i = 0; i < VPT; ++i) {
       const int c = threadIdx.x + i * LN_THREADS;
-      if (c < nv) qr[c] = quant4(v[i], inv);
+      if (c < nv) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
     }
-    if (threadIdx.x == 0) row_scale[row] = __fdiv_rn(amax, E4M3_MAX);
+    const float mean = block_reduce_1sync<false>(s, red[k++ & 1]) / (float)D;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = threadIdx.x + i * LN_THREADS;
+      if (c < nv) {
+        const float a = v[i].x - mean, b = v[i].y - mean, cc = v[i].z - mean, d = v[i].w - mean;
+        ss += (a * a + b * b) + (cc * cc + d * d);
+      }
+    }
+    const float var = block_reduce_1sync<false>(ss, red[k++ & 1]) / (float)D;
+    const float rstd = 1.0f / sqrtf(var + eps);
+    const float *mshift = nullptr, *mscale = nullptr, *bshift = nullptr, *bscale = nullptr;
+    if (md.mod) {
+      const float *mrow = md.mod + (size_t)(row / md.rows_div) * md.row_stride;
+      mshift = mrow + md.shift_off;
+      mscale = mrow + md.scale_off;
+      if (md.bias) {
+        bshift = md.bias + md.bias_shift_off;
+        bscale = md.bias + md.bias_scale_off;
+      }
+    }
+    OutT *orow = out + (size_t)row * D;
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int c = threadIdx.x + i * LN_THREADS;
+      if (c < nv) {
+        float4 u = make_float4((v[i].x - mean) * rstd, (v[i].y - mean) * rstd,
+                               (v[i].z - mean) * rstd, (v[i].w - mean) * rstd);
+        float4 a, b;
+        if (md.mod) {
+          float4 sc = load4(mscale + 4 * c), sh = load4(mshift + 4 * c);
+          if (bshift) {
+            const float4 bs = load4(bscale + 4 * c), bh = load4(bshift + 4 * c);
+            sc = make_float4(sc.x + bs.x, sc.y + bs.y, sc.z + bs.z, sc.w + bs.w);
+            sh = make_float4(sh.x + bh.x, sh.y + bh.y, sh.z + bh.z, sh.w + bh.w);
+          }
+          a = make_float4(1.f + sc.x, 1.f + sc.y, 1.f + sc.z, 1.f + sc.w);
+          b = sh;
+        } else {
+          a = load4(g + 4 * c);
+          b = load4(beta + 4 * c);
+        }
+        u.x = fmaf(u.x, a.x, b.x);
+        u.y = fmaf(u.y, a.y, b.y);
+        u.z = fmaf(u.z, a.z, b.z);
+        u.w = fmaf(u.w, a.w, b.w);
+        if constexpr (sizeof(OutT) == 1) {
+          v[i] = u;
+          amax = fmaxf(amax, absmax4(u));
+        } else {
+          store4(orow + 4 * c, u);
+        }
+      }
+    }
+    if constexpr (sizeof(OutT) == 1) {
+      amax = block_reduce_1sync<true>(amax, red[k++ & 1]);
+      const float inv = e4m3_inv_scale(amax);
+      uint32_t *qr = reinterpret_cast<uint32_t *>(orow);
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const int c = threadIdx.x + i * LN_THREADS;
+        if (c < nv) qr[c] = quant4(v[i], inv);
+      }
+      if (threadIdx.x == 0) row_scale[row] = __fdiv_rn(amax, E4M3_MAX);
+    }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) v[i] = nxt[i];
+  }
+}
+
+template <typename OutT, int VPT>
+static void ln_launch(const float *x, OutT *out, int rows, int D, const LnMod &m, const float *g,
+                      const float *beta, float eps, float *row_scale, cudaStream_t s) {
+  const int grid = rows < LN_CTAS_PER_SM * sm_count() ? rows : LN_CTAS_PER_SM * sm_count();
+  layernorm_mod_kernel<OutT, VPT><<<grid, LN_THREADS, 0, s>>>(x, out, rows, D, m, g, beta, eps, row_scale);
+}
+
+template <typename OutT>
+static void ln_dispatch(const float *x, OutT *out, int rows, int D, const LnMod &m, const float *g,
+                        const float *beta, float eps, float *row_scale, cudaStream_t s) {
+  switch ((D / 4 + LN_THREADS - 1) / LN_THREADS) {
+    case 1: ln_launch<OutT, 1>(x, out, rows, D, m, g, beta, eps, row_scale, s); break;
+    case 2: ln_launch<OutT, 2>(x, out, rows, D, m, g, beta, eps, row_scale, s); break;
+    case 3: ln_launch<OutT, 3>(x, out, rows, D, m, g, beta, eps, row_scale, s); break;
+    case 4: ln_launch<OutT, 4>(x, out, rows, D, m, g, beta, eps, row_scale, s); break;
+    case 5: ln_launch<OutT, 5>(x, out, rows, D, m, g, beta, eps, row_scale, s); break;
+    case 6: ln_launch<OutT, 6>(x, out, rows, D, m, g, beta, eps, row_scale, s); break;
+    default: ln_launch<OutT, LN_MAXV>(x, out, rows, D, m, g, beta, eps, row_scale, s); break;
   }
 }
 
@@ -304,9 +370,9 @@ int launch_layernorm_mod(const float *x, void *out, int dtype, int rows, int D, 
   if (D % 4 || D > 4 * LN_MAXV * LN_THREADS) return set_error(WAN_EUNSUPPORTED, "layernorm: D=%d", D);
   if (rows == 0) return WAN_OK;
   if (dtype == WAN_BF16)
-    layernorm_mod_kernel<__nv_bfloat16><<<rows, LN_THREADS, 0, s>>>(x, (__nv_bfloat16 *)out, D, m, g, beta, eps, nullptr);
+    ln_dispatch<__nv_bfloat16>(x, (__nv_bfloat16 *)out, rows, D, m, g, beta, eps, nullptr, s);
   else
-    layernorm_mod_kernel<float><<<rows, LN_THREADS, 0, s>>>(x, (float *)out, D, m, g, beta, eps, nullptr);
+    ln_dispatch<float>(x, (float *)out, rows, D, m, g, beta, eps, nullptr, s);
   WAN_CHECK_LAUNCH("layernorm_mod");
   return WAN_OK;
 }
@@ -315,7 +381,7 @@ int launch_layernorm_mod_fp8(const float *x, uint8_t *q, float *row_scale, int r
                              const float *g, const float *beta, float eps, cudaStream_t s) {
   if (D % 4 || D > 4 * LN_MAXV * LN_THREADS) return set_error(WAN_EUNSUPPORTED, "layernorm: D=%d", D);
   if (rows == 0) return WAN_OK;
-  layernorm_mod_kernel<uint8_t><<<rows, LN_THREADS, 0, s>>>(x, q, D, m, g, beta, eps, row_scale);
+  ln_dispatch<uint8_t>(x, q, rows, D, m, g, beta, eps, row_scale, s);
   WAN_CHECK_LAUNCH("layernorm_mod_fp8");
   return WAN_OK;
 }

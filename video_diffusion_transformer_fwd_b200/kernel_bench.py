@@ -5,6 +5,7 @@ driver used for ncu captures of one kernel on a small case).
     python -m video_diffusion_transformer_fwd_b200.kernel_bench block --config a14b-step --B 2
     python -m video_diffusion_transformer_fwd_b200.kernel_bench block --config a14b-step --F 5 ...
     python -m video_diffusion_transformer_fwd_b200.kernel_bench model --blocks 0
+    python -m video_diffusion_transformer_fwd_b200.kernel_bench euler --n 33554432
 
 Prints one JSON line with the mean device time per call (CUDA events on the
 launching stream, after warm-up) and the per-kernel-class times.
@@ -40,7 +41,8 @@ def _time(fn, iters, warmup):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["attention", "block", "model"])
+    ap.add_argument("what", choices=["attention", "block", "model", "euler"])
+    ap.add_argument("--n", type=int, default=1 << 25, help="euler: elements of the token state")
     ap.add_argument("--blocks", type=int, default=0)
     ap.add_argument("--fp8", action="store_true", help="block: FP8 GEMM mode")
     ap.add_argument("--attn8", action="store_true", help="8-bit attention (block: with FP8 GEMMs)")
@@ -68,6 +70,13 @@ def main():
         flops = 4.0 * a.B * a.L * Lk * a.heads * 128
         print(json.dumps({"what": "attention", "attn8": a.attn8, "B": a.B, "Lq": a.L, "Lk": Lk, "heads": a.heads,
                           "ms": ms, "tflops": flops / ms / 1e9, "kernels_ms": prof}))
+        return
+    if a.what == "euler":
+        # CFG + Euler on fp32 state and velocities: 16 bytes of HBM traffic per element
+        g = torch.Generator(device="cuda").manual_seed(7)
+        x, vc, vu = (torch.randn(a.n, device="cuda", generator=g) for _ in range(3))
+        ms, prof = _time(lambda: wan.euler_cfg_step(x, vc, vu, 5.0, 0.9, 0.875), a.iters, a.warmup)
+        print(json.dumps({"what": "euler", "n": a.n, "ms": ms, "gbs": 16.0 * a.n / ms / 1e6, "kernels_ms": prof}))
         return
     cfg = configs.get(a.config)
     if a.what == "model":
