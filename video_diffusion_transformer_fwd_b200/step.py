@@ -60,6 +60,86 @@ class DenoiseStep:
         return self.x
 
 
+
+def cfg_pairs(world: int):
+    """Rank pairs of the CFG-parallel step: ranks 2p and 2p + 1 run the
+    conditional and the unconditional branch of one denoising step."""
+    if world < 2 or world % 2:
+        raise ValueError(f"the CFG-parallel step needs an even number of ranks, got {world}")
+    return [[2 * p, 2 * p + 1] for p in range(world // 2)]
+
+
+def cfg_exchange(local, gathered, group):
+    """All-gather of the pair's two block outputs: ``local`` is this rank's
+    [1, L, D] output, ``gathered`` [2, L, D] receives the conditional one
+    (the pair's first rank) at 0 and the unconditional one at 1. NCCL writes
+    straight into ``gathered`` (over NVLink between GPUs of one node); other
+    backends gather into its two rows."""
+    import torch.distributed as dist
+    if dist.get_backend(group) == "nccl":
+        dist.all_gather_into_tensor(gathered, local, group=group)
+    else:
+        dist.all_gather([gathered[0], gathered[1]], local[0], group=group)
+
+
+class CFGParallelStep:
+    """The denoising step of DenoiseStep with the CFG pair split over two
+    ranks (two GPUs): each rank runs the block stack on its branch alone
+    (B = 1, its own context, the shared x and timestep), the two block
+    outputs are exchanged within the pair, and each rank applies
+    wan_euler_cfg_step to its own copy of x, so both copies stay equal. With
+    the same seed the inputs and weights are those of DenoiseStep, and since
+    no kernel mixes sequences, each rank's branch output equals that
+    sequence of the batched step.
+
+    ``branch`` 0 = conditional, 1 = unconditional (the rank's index within
+    ``group``, a process group of the two ranks)."""
+
+    def __init__(self, cfg: BlockConfig, branch: int, group, seed: int = 0, device: str = "cuda",
+                 weights=None):
+        if branch not in (0, 1):
+            raise ValueError(f"branch must be 0 (conditional) or 1 (unconditional), got {branch}")
+        self.cfg = cfg
+        self.branch = branch
+        self.group = group
+        self.dims = wan.dims_of(cfg)
+        self.device = device
+        self.weights = weights if weights is not None else synth.step_weights(cfg, device, seed)
+        self.cweights = [wan.make_weights(w) for w in self.weights]
+        acts = synth.block_activations(2, cfg.L, cfg.dim, cfg.text_len, cfg.dtype, device,
+                                       seed + 100, same_e0=True)
+        self.x = acts["x"][0].contiguous()                              # [L, D] float32, the state
+        self.ctx = acts["ctx"][branch:branch + 1].contiguous()          # [1, T, D]: this branch
+        self.e0 = acts["e0"][branch:branch + 1].contiguous()            # [1, 6, D]
+        self.xb = torch.empty((1, cfg.L, cfg.dim), dtype=torch.float32, device=device)
+        self.v = torch.empty((2, cfg.L, cfg.dim), dtype=torch.float32, device=device)
+        self.rope = wan.rope_freqs(cfg.head_dim, 1024, cfg.theta, device=device)
+        self.ws = wan.alloc_workspace(self.dims, 1, device=device)
+        self.ws_bytes = self.ws.numel()
+
+    def blocks(self, stream=None):
+        """This branch's block stack on xb (in place)."""
+        s = wan._stream(stream)
+        for cw in self.cweights:
+            wan.check(wan.wan_block_forward(self.dims, 1, self.xb.data_ptr(), self.ctx.data_ptr(),
+                                            None, self.e0.data_ptr(), cw, self.rope.data_ptr(),
+                                            self.rope.shape[0], self.ws.data_ptr(), self.ws_bytes,
+                                            s))
+
+    def step(self, stream=None):
+        """One step; the copy, the blocks, the exchange and the update are
+        ordered on ``stream`` (a torch CUDA stream; default the current one)."""
+        c = self.cfg
+        stream = stream if stream is not None else torch.cuda.current_stream()
+        with torch.cuda.stream(stream):
+            self.xb[0].copy_(self.x)
+            self.blocks(stream)
+            cfg_exchange(self.xb, self.v, self.group)
+            wan.check(wan.wan_euler_cfg_step(self.x.data_ptr(), self.v[0].data_ptr(), self.v[1].data_ptr(),
+                                             wan.WAN_F32, self.x.numel(), c.guide_scale, c.sigma,
+                                             c.sigma_next, wan._stream(stream)))
+        return self.x
+
 class ModelDenoiseStep:
     """One CFG flow-matching Euler step on the latent through the whole model
     (wan_model_forward on the CFG pair at t = 1000 sigma, then
