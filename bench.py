@@ -141,7 +141,7 @@ class OracleSample:
     fixed per-call cost of the text K/V projection). Inputs are drawn once
     by the seeded generators; only the oracle calls are timed."""
 
-    def __init__(self, cfg, seed=0, r_kv=4096, r_q=8, fp8=False):
+    def __init__(self, cfg, seed=0, r_kv=4096, r_q=12, fp8=False):
         import numpy as np
 
         from video_diffusion_transformer_fwd_b200 import synth

@@ -220,6 +220,15 @@ def test_block_bf16_small_sharp():
     _bf16_block_check(cfg, B=2, gain_scale=4.0)
 
 
+@pytest.mark.parametrize("dim", [4096, 7168, 8192])
+def test_block_bf16_wide_dims(dim):
+    """Model widths beyond the configs' (up to the LayerNorm's 8192 limit): every
+    row layout of the LayerNorm kernel (float4 chunks per thread: 4, 7 and 8)
+    and head counts 32 to 64, on a small ragged token grid."""
+    cfg = BlockConfig(f"bf16-wide-{dim}", 2, 3, 5, dim, dim // 128, dim, 16, "bf16")
+    _bf16_block_check(cfg, B=2, ctx_lens=[16, 5])
+
+
 def test_block_1p3b_short():
     _bf16_block_check(configs.get("1.3b-short"))
 
