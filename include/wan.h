@@ -158,7 +158,12 @@ size_t wan_block_workspace_offset(const wan_dims *dims, int B, int which);
  *
  *   dims      problem statement; head_dim must be 128 for WAN_BF16 and
  *             WAN_FP8, and one of 32, 64, 128 for WAN_F32. dim % 64 == 0,
- *             ffn_dim % 64 == 0 (WAN_FP8: dim % 256 == 0, ffn_dim % 128 == 0).
+ *             ffn_dim % 64 == 0; WAN_BF16 and WAN_FP8 also need
+ *             dim % 256 == 0 (WAN_FP8: ffn_dim % 128 == 0).
+ *             The dtype picks the kernels: WAN_F32 runs every product on
+ *             the exact-fp32 CUDA-core kernels, WAN_BF16 / WAN_FP8 on the
+ *             tcgen05 tensor-core kernels; a shape outside a kernel's rules
+ *             is refused with WAN_EUNSUPPORTED, never run on another kernel.
  *   B         sequences (2 for a CFG pair: same x, two contexts), >= 1.
  *   x         in/out float32 [B, L, dim], the residual stream.
  *   ctx       (dt) [B, T, dim] projected text tokens.
@@ -191,8 +196,10 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx,
  *   holds until the process exits; the entry point itself allocates nothing.
  *   Problems with wan_block_workspace_bytes(dims, B) above that size are
  *   rejected (WAN_EINVAL, message names both sizes).
- *   The array's device address is looked up on the first call made with a
- *   given device current: make that first call before any stream capture.
+ *   The array's device address is looked up on every call made while the
+ *   stream is not capturing (a device reset moves the array); the first call
+ *   with a given device current must come before any stream capture.
+ *   B == 0 and invalid dims give the same status as wan_block_forward.
  *   All calls on a device share the array and it keeps the previous call's
  *   contents (the block writes every byte it reads, so no clearing is
  *   needed); calls that may overlap on the GPU race on it. */
@@ -257,6 +264,11 @@ size_t wan_model_workspace_bytes(const wan_model_dims *dims, int B);
  * Constraints: wan_dims rules for the token grid (F, H/2, W/2) and dim / heads /
  * ffn_dim; H, W even; C_in * 4 and freq_dim multiples of 8; text_dim a multiple
  * of 64 (when text_len > 0); num_blocks >= 0; every pointer 16-byte aligned.
+ * Kernels: the blocks as in wan_block_forward; the time MLP (fp32, B rows)
+ * on a small-M weight-streaming kernel; with WAN_BF16 the patch embedding,
+ * text MLP and head on the tensor-core GEMM, except a patch embedding whose
+ * 4 * C_in is not a multiple of 64 (I2V's 36 channels), which runs on the
+ * CUDA-core GEMM (K = 144: a negligible share of the model's work).
  * The workspace holds the token stream, the embeddings and one block
  * workspace; the head's normalised tokens reuse the block's ACT buffer.
  * Errors: as wan_block_forward. */

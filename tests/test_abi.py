@@ -115,3 +115,35 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert wan.wan_euler_cfg_step(None, 32, None, wan.WAN_F32, 10, 5.0, 0.9, 0.875, None) == wan.WAN_EINVAL
     assert wan.wan_euler_cfg_step(16, 32, None, 5, 10, 5.0, 0.9, 0.875, None) == wan.WAN_EUNSUPPORTED
     assert wan.wan_euler_cfg_step(18, 32, None, wan.WAN_F32, 10, 5.0, 0.9, 0.875, None) == wan.WAN_EALIGN
+
+
+def test_noalloc_array_size_matches_header():
+    """The binding's copy of WAN_NOALLOC_WORKSPACE_BYTES is the header's."""
+    src = open(os.path.join(ROOT, "include", "wan.h")).read()
+    m = re.search(r"#define\s+WAN_NOALLOC_WORKSPACE_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", src)
+    assert m, "define not found"
+    assert int(m.group(1)) << int(m.group(2)) == wan.WAN_NOALLOC_WORKSPACE_BYTES
+
+
+def test_noalloc_empty_and_invalid_calls_match_the_workspace_entry_point(lib):
+    """B == 0 and invalid dims give wan_block_forward's status and message."""
+    w = wan.wan_block_weights(*([4096] * len(wan.WEIGHT_FIELDS)))
+    for d, B in ((dims(), 0), (dims(dim=100), 0), (dims(dim=100), 1), (dims(dtype="bf16"), 1),
+                 (dims(), -1)):
+        rc_ws = wan.wan_block_forward(d, B, 16, 16, None, 16, w, 16, 1024, 16, 1 << 30, None)
+        msg_ws = wan.last_error()
+        rc_na = wan.wan_block_forward_noalloc(d, B, 16, 16, None, 16, w, 16, 1024, None)
+        assert rc_na == rc_ws, (B, rc_na, rc_ws)
+        assert wan.last_error() == msg_ws
+
+
+@pytest.mark.parametrize("kw", [dict(dim=384, heads=3, ffn_dim=512), dict(dim=640, heads=5, ffn_dim=512)])
+def test_bf16_block_outside_tensor_core_rules_is_refused(lib, kw):
+    """A bf16 block whose dim is not a multiple of 256 cannot use the
+    tensor-core QKV epilogue; it is refused, never run on other kernels."""
+    d = dims(dtype="bf16", **kw)
+    w = wan.wan_block_weights(*([4096] * len(wan.WEIGHT_FIELDS)))
+    rc = wan.wan_block_forward(d, 1, 16, 16, None, 16, w, 16, 1024, 16, 1 << 40, None)
+    assert rc == wan.WAN_EUNSUPPORTED
+    assert "256" in wan.last_error()
+    assert wan.wan_block_workspace_bytes(d, 1) == 0

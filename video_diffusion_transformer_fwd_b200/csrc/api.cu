@@ -47,15 +47,30 @@ int *watchdog_ptr() {
 }
 
 // ---------------------------------------------------------------- dispatch
+// The kernel is chosen by dtype alone: WAN_F32 runs the exact-fp32 CUDA-core
+// kernels, WAN_BF16 the tcgen05 tensor-core kernels. A bf16 problem outside
+// the tensor-core kernels' shape rules is refused (WAN_EUNSUPPORTED, with the
+// rule in the message); it never falls back to another kernel.
 static int run_gemm(const GemmArgs &g, int dtype, cudaStream_t s) {
-  if (dtype == WAN_BF16 && gemm_tc_supported(g)) return WAN_PROF(WAN_K_GEMM_TC, s, gemm_tc(g, s));
-  return WAN_PROF(WAN_K_GEMM_SIMT, s, gemm_simt(g, dtype, s));
+  if (dtype == WAN_F32) return WAN_PROF(WAN_K_GEMM_SIMT, s, gemm_simt(g, dtype, s));
+  if (dtype != WAN_BF16) return set_error(WAN_EUNSUPPORTED, "GEMM dtype %d", dtype);
+  if (!gemm_tc_supported(g))
+    return set_error(WAN_EUNSUPPORTED,
+                     "bf16 GEMM M=%d N=%d K=%d outside the tensor-core kernel's rules (K %% 64 == 0, N %% 32 == 0, "
+                     "256-column weight segments, 16-byte aligned rows)", g.M, g.N, g.K);
+  return WAN_PROF(WAN_K_GEMM_TC, s, gemm_tc(g, s));
 }
 
-// cls: profiling class used when the tensor-core kernel runs
+// cls: profiling class of the tensor-core launch
 static int run_attention(const AttnArgs &a, int dtype, cudaStream_t s, int cls) {
-  if (dtype == WAN_BF16 && attention_tc_supported(a)) return WAN_PROF(cls, s, attention_tc(a, s));
-  return WAN_PROF(WAN_K_ATTN_SIMT, s, attention_simt(a, dtype, s));
+  if (dtype == WAN_F32) return WAN_PROF(WAN_K_ATTN_SIMT, s, attention_simt(a, dtype, s));
+  if (dtype != WAN_BF16) return set_error(WAN_EUNSUPPORTED, "attention dtype %d", dtype);
+  if (!attention_tc_supported(a))
+    return set_error(WAN_EUNSUPPORTED,
+                     "bf16 attention (B=%d heads=%d Lq=%d Lk=%d d=%d) outside the tensor-core kernel's rules "
+                     "(head_dim 128, row strides %% 8 == 0, 16-byte aligned, B and heads <= 65535)",
+                     a.B, a.heads, a.Lq, a.Lk, a.d);
+  return WAN_PROF(cls, s, attention_tc(a, s));
 }
 
 // ---------------------------------------------------------------- workspace
@@ -103,8 +118,11 @@ static int check_dims(const wan_dims *d, int B) {
     return set_error(WAN_EUNSUPPORTED, "dtype %d", d->dtype);
   const int hd = d->dim / d->heads;
   if (d->dtype != WAN_F32 && hd != 128) return set_error(WAN_EUNSUPPORTED, "bf16 / fp8 paths need head_dim 128 (got %d)", hd);
-  if (is_fp8(d->dtype) && (d->dim % 256 || d->ffn_dim % 128))
-    return set_error(WAN_EUNSUPPORTED, "fp8 path needs dim %% 256 == 0 and ffn_dim %% 128 == 0");
+  if (d->dtype != WAN_F32 && d->dim % 256)
+    return set_error(WAN_EUNSUPPORTED, "bf16 / fp8 paths need dim %% 256 == 0 (got %d): the QKV epilogue "
+                                       "normalises q and k over whole 256-column tiles", d->dim);
+  if (is_fp8(d->dtype) && d->ffn_dim % 128)
+    return set_error(WAN_EUNSUPPORTED, "fp8 path needs ffn_dim %% 128 == 0");
   if (d->dtype == WAN_F32 && hd != 32 && hd != 64 && hd != 128)
     return set_error(WAN_EUNSUPPORTED, "fp32 path needs head_dim 32, 64 or 128 (got %d)", hd);
   const long long L = (long long)d->F * d->H * d->W;
@@ -371,7 +389,10 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
   aself.B = B; aself.heads = d.heads; aself.Lq = L; aself.Lk = L; aself.d = hd;
   aself.q = qkv; aself.ldq = 3 * D; aself.k = qkv + D * es; aself.ldk = 3 * D; aself.v = qkv + 2 * D * es; aself.ldv = 3 * D;
   aself.o = o; aself.ldo = D; aself.k_lens = nullptr; aself.scale = 1.0f / sqrtf((float)hd);
-  const bool fused = dt == WAN_BF16 && gemm_tc_supported(gqkv) && attention_tc_supported(aself);
+  const bool fused = dt == WAN_BF16;
+  if (fused && !(gemm_tc_supported(gqkv) && attention_tc_supported(aself)))
+    return set_error(WAN_EUNSUPPORTED, "bf16 block: the QKV GEMM or the self-attention is outside the "
+                                       "tensor-core kernels' rules (dim %% 256 == 0, head_dim 128)");
 
   if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, ln_of(ms, 0, 1), nullptr, nullptr, d.eps, s)))) return rc;
   if (fused) {

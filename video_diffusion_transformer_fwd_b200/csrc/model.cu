@@ -132,10 +132,20 @@ ModelLayout model_layout(const wan_model_dims &m, int B) {
   return l;
 }
 
-int gemm_any(const GemmArgs &g, int dtype, cudaStream_t s) {
+// Kernel choice for the model's own GEMMs, by shape and dtype, never as a
+// silent fallback: a few rows (the time MLP at M = B) stream the weight once
+// in the small-M kernel; fp32 runs the exact CUDA-core GEMM; bf16 runs the
+// tensor-core GEMM, except the patch embedding when 4 * C_in is not a
+// multiple of 64 (the I2V input's 36 channels: K = 144), which is documented
+// to run on the CUDA-core GEMM (`small_k_on_cuda_cores`). Any other bf16 shape
+// outside the tensor-core rules is refused.
+int gemm_any(const GemmArgs &g, int dtype, cudaStream_t s, bool small_k_on_cuda_cores = false) {
   if (gemm_smallm_supported(g)) return WAN_PROF(WAN_K_MODEL, s, gemm_smallm(g, dtype, s));
-  if (dtype == WAN_BF16 && gemm_tc_supported(g)) return WAN_PROF(WAN_K_GEMM_TC, s, gemm_tc(g, s));
-  return WAN_PROF(WAN_K_GEMM_SIMT, s, gemm_simt(g, dtype, s));
+  if (dtype == WAN_F32) return WAN_PROF(WAN_K_GEMM_SIMT, s, gemm_simt(g, dtype, s));
+  if (gemm_tc_supported(g)) return WAN_PROF(WAN_K_GEMM_TC, s, gemm_tc(g, s));
+  if (small_k_on_cuda_cores && g.K % 64) return WAN_PROF(WAN_K_GEMM_SIMT, s, gemm_simt(g, dtype, s));
+  return set_error(WAN_EUNSUPPORTED, "model bf16 GEMM M=%d N=%d K=%d outside the tensor-core kernel's rules "
+                                     "(K %% 64 == 0, N %% 32 == 0)", g.M, g.N, g.K);
 }
 
 }  // namespace
@@ -211,7 +221,7 @@ int wan_model_forward(const wan_model_dims *dims, int B, const float *latent, co
     g.Bseg[0] = w->patch_w; g.bias[0] = w->patch_b; g.segN = D; g.nseg = 1;
     g.epi = EPI_RESID; g.X = X; g.ldx = D; g.gate = nullptr; g.rows_per_gate = L;
     g.x_store = 1;
-    if ((rc = gemm_any(g, dt, s))) return rc;
+    if ((rc = gemm_any(g, dt, s, /*small_k_on_cuda_cores=*/true))) return rc;
   }
   // time embedding (fp32): e = W2 SiLU(W1 sinusoid(t) + b1) + b2; e0 = Wp SiLU(e) + bp,
   // for B timesteps or, per token, B * L
