@@ -299,18 +299,19 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
 
 # --------------------------------------------------------------------------
 # 8-bit attention ([DIGEST] inference-optimisation table, "8-bit
-# FlashAttention": int8 for S = Q K^T, FP8 for O = P V, fp32 accumulation
-# across key blocks). Readings where the page is silent: q is quantized per
-# token and head (scale amax/127 over the head's d values), k per head over
-# all keys of the sequence, v to e4m3 per head and channel over all keys
-# (the channel scale factors out of P V). Keys are taken in blocks of 128 in
-# order, FlashAttention style, in log2 units t = s log2(e): a row keeps a
-# frame F, the running max rounded up to a multiple of 8, raised after a
-# block whenever that block's max exceeds it (the earlier sum and output are
-# then rescaled by 2^(F_old - F)); the block's P = 2^(t - F + 8) lies in
-# (0, 2^8] and is rounded to e4m3 for the P V product; the row normaliser
-# sums the unrounded P. int8 codes are round-half-even of x * (127 / amax),
-# clamped to +-127, decided in fp32.
+# FlashAttention": int8 for S = Q K^T, FP8 for O = P V, fp32 accumulation).
+# The page gives only the types, so this is the plain definition with each
+# product's operands quantized: S from int8 q and k (exact integer products
+# times the two scales and the logit scale), the softmax probabilities
+# p = exp(s - m) with m the exact row max over the valid keys, and O = P V
+# with P and V in e4m3. Readings where the page is silent: q is quantized per
+# token and head (scale amax / 127 over the head's d values), k per head over
+# all keys of the sequence, v to e4m3 per head and channel over all keys (the
+# channel scale factors out of P V); P by the FP8 rule of the GEMMs (one
+# scale per row = amax / 448, and the row's amax is p = 1 at the max, so the
+# codes are e4m3(448 p)); the normaliser sums the unrounded p. int8 codes
+# are round-half-even of x * (127 / amax), clamped to +-127, decided in fp32.
+# Sums are exact (fp64); no blocking or running max.
 # --------------------------------------------------------------------------
 I8_MAX = 127.0
 
@@ -339,11 +340,12 @@ def quantize_fp8_axes(x, axes):
     return e4m3_round(y.astype(F64)), (amax / np.float32(E4M3_MAX)).astype(np.float32).astype(F64)
 
 
-def attention_8bit(q, k, v, k_len: int | None = None, scale: float | None = None,
-                   block: int = 128) -> np.ndarray:
-    """8-bit softmax attention of one sequence (q [Lq, n, d], k, v [Lk, n, d];
-    the first ``k_len`` keys valid). The scales of k and v are taken over all
-    Lk keys; keys are visited in blocks of ``block``."""
+def attention_8bit_terms(q, k, v, k_len: int | None = None, scale: float | None = None):
+    """The quantities the 8-bit attention of one sequence is formed from
+    (q [Lq, n, d], k, v [Lk, n, d]; the first ``k_len`` keys valid):
+    p [n, Lq, kl] = exp(s - rowmax s) over the valid keys, with s the
+    quantized logits; l [n, Lq, 1] = sum of p; vq [kl, n, d] the e4m3 codes
+    of v and sv [1, n, d] their per-channel scales."""
     q = np.asarray(q, F64)
     k = np.asarray(k, F64)
     v = np.asarray(v, F64)
@@ -354,23 +356,26 @@ def attention_8bit(q, k, v, k_len: int | None = None, scale: float | None = None
     ki, sk = quantize_int8(k, axes=(0, 2))         # [1, n, 1]
     vq, sv = quantize_fp8_axes(v, axes=(0,))       # [1, n, d]
     kl = k.shape[0] if k_len is None else k_len
-    c = np.transpose(sq, (1, 0, 2)) * sk[0][:, :, None] * scale / math.log(2.0)    # [n, Lq, 1]
-    frame = np.full((n, Lq, 1), -np.inf)
-    l = np.zeros((n, Lq, 1))
-    o = np.zeros((n, Lq, d))
-    for j0 in range(0, kl, block):
-        j1 = min(j0 + block, kl)
-        t = np.einsum("qnd,knd->nqk", qi, ki[j0:j1]) * c            # exact integer products, log2 units
-        tmax = t.max(-1, keepdims=True)
-        f_new = np.where(tmax > frame, 8.0 * np.ceil(tmax / 8.0), frame)
-        corr = np.exp2(frame - f_new)                                  # 0 on the first block
-        p = np.exp2(t - f_new + 8.0)
-        l = l * corr + p.sum(-1, keepdims=True)
-        o = o * corr + np.einsum("nqk,knd->nqd", e4m3_round(p), vq[j0:j1])
-        frame = f_new
+    s = np.einsum("qnd,knd->nqk", qi, ki[:kl]) * (np.transpose(sq, (1, 0, 2)) * sk[0][:, :, None] * scale)
     if kl == 0:
+        return np.zeros((n, Lq, 0)), np.zeros((n, Lq, 1)), vq[:0], sv
+    p = np.exp(s - s.max(-1, keepdims=True))
+    return p, p.sum(-1, keepdims=True), vq[:kl], sv
+
+
+def attention_8bit(q, k, v, k_len: int | None = None, scale: float | None = None) -> np.ndarray:
+    """8-bit softmax attention of one sequence (q [Lq, n, d], k, v [Lk, n, d];
+    the first ``k_len`` keys valid): o = (sum_j e4m3(448 p_j) / 448 vq_j) / l
+    times the channel scales of v. A row with no valid key returns zeros."""
+    Lq, n, d = np.shape(q)
+    p, l, vq, sv = attention_8bit_terms(q, k, v, k_len, scale)
+    if p.shape[2] == 0:
         return np.zeros((Lq, n, d), F64)
-    return np.transpose(o / l, (1, 0, 2)) * sv
+    pq = e4m3_round(p * E4M3_MAX) / E4M3_MAX
+    o = np.einsum("nqk,knd->nqd", pq, vq) / l
+    return np.transpose(o, (1, 0, 2)) * sv
+
+
 # --------------------------------------------------------------------------
 # The block ([WALK] WanAttentionBlock core-logic snippet; [DIGEST] shared
 # AdaLN MLP + per-block bias)

@@ -1,7 +1,8 @@
 """Pins of the oracle's 8-bit attention ("Wan paper deep dive",
 inference-optimisation table, "8-bit FlashAttention": int8 S = Q K^T, FP8
 O = P V): the int8 quantizer's invariants, exactness when every
-quantization step is the identity, how each scale enters, and the size of the
+quantization step is the identity, P relative to the exact row max, no
+dependence on key order, how each scale enters, and the size of the
 approximation."""
 import math
 
@@ -59,10 +60,45 @@ def test_attention_8bit_exact_when_quantization_is_identity():
         got = O.attention_8bit(q, k, v, k_len=kl, scale=ln2)
         ref = O.attention(q, k, v, k_len=kl, scale=ln2)
         assert np.abs(got - ref).max() <= 1e-12 * np.abs(ref).max()
-    # the key blocks only change where P is rounded: with every P a power of
-    # two the block size does not matter
-    assert np.abs(O.attention_8bit(q, k, v, scale=ln2, block=7) - O.attention_8bit(q, k, v, scale=ln2)).max() \
-        <= 1e-12 * np.abs(ref).max()
+
+
+def test_attention_8bit_p_is_relative_to_the_exact_row_max():
+    """P is exp(s - m) with m the row's exact maximum, quantized as 448 p:
+    the probability at the max is exactly 1 (code 448), so a single valid key
+    returns that key's dequantized value exactly, and a key whose logit is
+    ln(2) * j below the max carries weight 2^-j exactly while 448 * 2^-j is
+    an e4m3 value (j <= 15)."""
+    rng = np.random.default_rng(4)
+    q, k, v = (rng.standard_normal((9, 2, 128)) for _ in range(3))
+    vq, sv = O.quantize_fp8_axes(v, axes=(0,))
+    one = O.attention_8bit(q, k, v, k_len=1)
+    assert np.array_equal(one, np.broadcast_to(vq[0] * sv[0], one.shape))
+    # two keys: logits 0 and -j ln 2 exactly (int8 codes, scale ln 2)
+    for j in (1, 5, 15):
+        qq = np.zeros((1, 1, 128))
+        kk = np.zeros((2, 1, 128))
+        qq[0, 0, 0] = 127.0
+        kk[0, 0, 1] = 127.0                  # logit 0 (orthogonal), amax of k = 127
+        kk[1, 0, 0] = -float(j)              # logit -127 j: with scale ln2 / 127, -j ln 2
+        vv = np.zeros((2, 1, 128))
+        vv[0, 0, :] = 448.0
+        vv[1, 0, :] = -448.0
+        got = O.attention_8bit(qq, kk, vv, scale=math.log(2.0) / 127.0)
+        w = 2.0 ** -j
+        assert np.abs(got - (1.0 - w) / (1.0 + w) * 448.0).max() <= 1e-12 * 448.0
+
+
+def test_attention_8bit_is_invariant_to_key_order():
+    """No blocking and no running max: permuting the keys (with their values)
+    leaves every output unchanged up to fp64 summation order."""
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((16, 2, 128)) * 3.0
+    k = rng.standard_normal((700, 2, 128)) * 3.0
+    v = rng.standard_normal((700, 2, 128))
+    perm = rng.permutation(700)
+    a = O.attention_8bit(q, k, v)
+    b = O.attention_8bit(q, k[perm], v[perm])
+    assert np.abs(a - b).max() <= 1e-12 * np.abs(a).max()
 
 
 def test_attention_8bit_scales_enter_where_they_should():
@@ -91,9 +127,14 @@ def test_attention_8bit_approximates_attention():
     err = np.linalg.norm(O.attention_8bit(q, k, v) - ref) / np.linalg.norm(ref)
     assert 1e-3 < err < 0.08
     assert not O.attention_8bit(q, k, v, k_len=0).any()
-    # one block holding every key: P is relative to the final row max
-    one = O.attention_8bit(q, k, v, block=256)
-    assert 1e-3 < np.linalg.norm(one - ref) / np.linalg.norm(ref) < 0.08
+    # the only approximations are the quantizers: with P unrounded (the terms'
+    # p) the result is attention over the int8 / e4m3 inputs exactly
+    p, l, vq, sv = O.attention_8bit_terms(q, k, v)
+    qi, sq = O.quantize_int8(q, axes=(2,))
+    ki, sk = O.quantize_int8(k, axes=(0, 2))
+    deq = O.attention(qi * sq, ki * sk, vq * sv)
+    unrounded = np.transpose(np.einsum("nqk,knd->nqd", p, vq) / l, (1, 0, 2)) * sv
+    assert np.abs(unrounded - deq).max() <= 1e-12 * np.abs(deq).max()
 
 
 def test_block_with_8bit_attention_close_to_fp8_block():
