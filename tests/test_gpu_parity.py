@@ -123,6 +123,18 @@ def test_block_tiny_f32_full():
     assert np.abs(run.ws_rows(wan.WAN_WS_H, TINY.ffn_dim, rows) - inter["h"]).max() <= F32_MAX_ABS
 
 
+def test_block_tiny_f32_against_scalar_oracle():
+    """The tiny fp32 block against the scalar-loop form of the oracle."""
+    from oracle import wan_oracle_scalar as S
+    run = GpuBlockRun(TINY, B=2, seed=0, ctx_lens=[8, 3]).run()
+    grid = (TINY.F, TINY.H, TINY.W)
+    w = weights64(run.w)
+    for b, kl in enumerate((8, 3)):
+        ref = np.array(S.block_forward(np64(run.x0[b]), np64(run.ctx[b]), kl, np64(run.e0[b]), w,
+                                       TINY.heads, grid, TINY.eps, TINY.theta))
+        assert np.abs(np64(run.x[b]) - ref).max() <= F32_MAX_ABS
+
+
 def test_block_tiny_f32_ctx_lens_and_sharp():
     run = GpuBlockRun(TINY, B=2, seed=3, ctx_lens=[5, 1], gain_scale=4.0).run()
     ref = run.oracle_rows(np.arange(TINY.L))
