@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--config", default="a14b-step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the single-block rows of the other configurations (run after the timed step)")
     ap.add_argument("--fp8", action="store_true",
                     help="FP8 GEMM mode of the blocks (e4m3 projections, bf16 attention); not the default")
     ap.add_argument("--attn8", action="store_true",
@@ -178,12 +180,77 @@ class OracleSample:
         per_row = max((times[1] - times[0]) / r_q, 0.0)
         fixed = max(times[0] - per_row * r_q, 0.0)
         est = t_kv * cfg.L / r_kv + fixed + per_row * cfg.L
-        detail = (("FP8-GEMM " if self.fp8 else "") + f"fp64 oracle on one block forward of the workload's block shape (one sequence): "
-                  f"LN + K/V projection timed on {r_kv} rows (scaled x{cfg.L / r_kv:.1f}); the rest "
-                  f"of the block timed for {r_q} and {2 * r_q} query rows attending over all {cfg.L} "
-                  f"keys (per-row cost x{cfg.L}, plus the per-call text K/V projection); "
-                  f"{t_kv + sum(times):.1f} s of CPU time sampled")
-        return est * 1e3, detail
+        detail = (("FP8-GEMM " if self.fp8 else "") + f"ESTIMATE from a measured sample: fp64 oracle on one block "
+                  f"forward of the workload's block shape (one sequence): LN + K/V projection timed on {r_kv} "
+                  f"rows (scaled x{cfg.L / r_kv:.1f}); the rest of the block timed for {r_q} and {2 * r_q} "
+                  f"query rows attending over all {cfg.L} keys (per-row cost x{cfg.L}, plus the per-call "
+                  f"text K/V projection); {t_kv + sum(times):.1f} s of CPU time sampled")
+        measured = {"kv_rows": r_kv, "kv_s": t_kv, "query_rows": [r_q, 2 * r_q], "query_s": times,
+                    "sampled_s": t_kv + sum(times)}
+        return est * 1e3, detail, measured
+
+
+def _oracle_rows_worker(args):
+    """One process of the full-block oracle run: the block at ``rows`` from
+    inputs memory-mapped from ``d`` (spawned, one BLAS thread)."""
+    d, heads, grid, eps, theta, rows = args
+    import numpy as np
+    try:
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+    except Exception:
+        pass
+    from oracle import wan_oracle as O
+    ld = lambda n: np.load(os.path.join(d, n + ".npy"), mmap_mode="r")
+    w = {k[2:]: ld(k) for k in (f[:-4] for f in os.listdir(d)) if k.startswith("w_")}
+    t0 = time.perf_counter()
+    out = O.block_forward_rows(ld("x"), ld("ctx"), None, ld("e0"), w, heads, grid, eps, rows,
+                               theta=theta, kv=(ld("k"), ld("v")))
+    return time.perf_counter() - t0, out.shape[1]
+
+
+def oracle_full_block(cfg, procs, seed=0):
+    """Un-extrapolated fp64 oracle time of one whole block forward of one
+    sequence of ``cfg``: the key / value projection of every row (the
+    oracle's self_attn_kv, multi-threaded BLAS), then block_forward_rows on
+    every row, the rows split over ``procs`` spawned processes. Only the
+    oracle calls are timed (inputs are drawn and shared beforehand)."""
+    import multiprocessing as mp
+    import shutil
+    import tempfile
+
+    import numpy as np
+
+    from oracle import wan_oracle as O
+    from video_diffusion_transformer_fwd_b200 import synth
+    w = synth.block_weights(cfg.dim, cfg.ffn_dim, cfg.dtype, "cpu", seed)
+    acts = synth.block_activations(1, cfg.L, cfg.dim, cfg.text_len, cfg.dtype, "cpu", seed + 100)
+    grid = (cfg.F, cfg.H, cfg.W)
+    d = tempfile.mkdtemp(prefix="wan_oracle_", dir="/dev/shm" if os.path.isdir("/dev/shm") else None)
+    try:
+        arr = {k: synth.to_numpy64(acts[k]) for k in ("x", "ctx", "e0")}
+        for k, v in w.items():
+            arr["w_" + k] = synth.to_numpy64(v)
+        t0 = time.perf_counter()
+        k, v = O.self_attn_kv(arr["x"], arr["e0"], {n[2:]: a for n, a in arr.items() if n.startswith("w_")},
+                              cfg.heads, grid, cfg.eps, cfg.theta)
+        t_kv = time.perf_counter() - t0
+        arr["k"], arr["v"] = k, v
+        for n, a in arr.items():
+            np.save(os.path.join(d, n + ".npy"), a)
+        chunks = [c for c in np.array_split(np.arange(cfg.L), procs) if len(c)]
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(len(chunks)) as pool:
+            pool.map(_oracle_rows_worker, [(d, cfg.heads, grid, cfg.eps, cfg.theta, chunks[0][:2])] * len(chunks))
+            t0 = time.perf_counter()
+            res = pool.map(_oracle_rows_worker, [(d, cfg.heads, grid, cfg.eps, cfg.theta, c) for c in chunks])
+            t_rows = time.perf_counter() - t0
+        assert sum(r[1] for r in res) == cfg.L
+        return {"config": cfg.name, "kind": "full block, every row (not extrapolated)", "rows": cfg.L,
+                "oracle_s": t_kv + t_rows, "kv_s": t_kv, "rows_s": t_rows, "processes": len(chunks),
+                "cpu_s": t_kv + sum(r[0] for r in res)}
+    finally:
+        shutil.rmtree(d, ignore_errors=True)
 
 
 def cpu_cores():
@@ -226,11 +293,11 @@ def run_reference(args, rank, world):
         return
     from video_diffusion_transformer_fwd_b200 import configs
     cfg = configs.get(args.config)
-    sample = OracleSample(cfg, seed=0)
+    sample = OracleSample(cfg, seed=0, r_kv=2048, r_q=8)
     vals = []
-    detail = ""
+    detail, measured = "", {}
     for i in range(args.warmup + args.steps):
-        ms, detail = sample.run()
+        ms, detail, measured = sample.run()
         if i >= args.warmup:
             vals.append(ms)
     value = statistics.mean(vals)
@@ -240,9 +307,10 @@ def run_reference(args, rank, world):
         "warmup": args.warmup, "ms_per_step": value * cfg.blocks * 2, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
+        "estimated": True,
         "config": workload_config(cfg, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "blas_threads": blas_threads(),
-                         "kind": "oracle", "sample": detail},
+                         "kind": "oracle", "estimated": True, "measured": measured, "sample": detail},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -261,6 +329,64 @@ def workload_config(cfg, world, cfg_parallel=False):
         "l2": "inputs larger than L2 (28 GB of block weights and a 671 MB token state per step)",
         "weights": "random N(0,0.02), synthetic x/ctx N(0,1)",
     }
+
+
+# ----------------------------------------------------------------- per-config block rows
+PER_CONFIG = (("1.3b-short", 1), ("1.3b-long", 1), ("5b", 1), ("a14b-step", 1), ("a14b-step", 2))
+
+
+def per_config_rows(dev, peaks, iters=5, warmup=2):
+    """One bf16 block forward per configuration of the workload table (random
+    N(0, 0.02) weights, x and ctx N(0, 1)), timed alone with CUDA events:
+    block ms and the attention / GEMM split from the per-launch events, with
+    fractions of the measured burst bf16 peak (kernels timed in isolation)."""
+    import dataclasses
+
+    import torch
+
+    from video_diffusion_transformer_fwd_b200 import configs, synth, wan
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    rows = []
+    stream = torch.cuda.current_stream()
+    for name, B in PER_CONFIG:
+        cfg = dataclasses.replace(configs.get(name), batch=B, blocks=1)
+        dims = wan.dims_of(cfg)
+        w = wan.make_weights(synth.block_weights(cfg.dim, cfg.ffn_dim, cfg.dtype, dev, 0))
+        acts = synth.block_activations(B, cfg.L, cfg.dim, cfg.text_len, cfg.dtype, dev, 100)
+        rope = wan.rope_freqs(cfg.head_dim, 1024, cfg.theta, device=dev)
+        ws = wan.alloc_workspace(dims, B, device=dev)
+        for _ in range(warmup):
+            wan.block_forward(dims, acts["x"], acts["ctx"], acts["e0"], w, rope, ws)
+        torch.cuda.synchronize()
+        clocks = ClockSampler([torch.cuda.current_device()])
+        wan.check(wan.wan_profile_enable(1))
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(iters):
+            wan.block_forward(dims, acts["x"], acts["ctx"], acts["e0"], w, rope, ws)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        prof = wan.profile_read()
+        wan.check(wan.wan_profile_enable(0))
+        ck = clocks.stop()
+        if wan.device_status() != wan.WAN_OK:
+            raise RuntimeError(f"per-config {name}: " + wan.last_error())
+        ms = t0.elapsed_time(t1) / iters
+        a_n, a_ms = prof["attn_self"]
+        g_n, g_ms = prof["gemm_tc"]
+        a_tf = cfg.self_attn_flops() * iters / (a_ms * 1e-3) / 1e12 if a_ms > 0 else None
+        g_tf = cfg.gemm_flops() * iters / (g_ms * 1e-3) / 1e12 if g_ms > 0 else None
+        rows.append({
+            "config": name, "B": B, "L": cfg.L, "dim": cfg.dim, "heads": cfg.heads, "ffn": cfg.ffn_dim,
+            "block_ms": ms, "block_tflops": cfg.block_flops() / (ms * 1e-3) / 1e12,
+            "attention_tflops": a_tf, "gemm_tflops": g_tf,
+            "attention_frac_of_measured_burst": None if a_tf is None else a_tf / burst,
+            "gemm_frac_of_measured_burst": None if g_tf is None else g_tf / burst,
+            "kernel_ms": {k: v[1] / iters for k, v in prof.items() if v[0]},
+            "clocks": {"sm_mhz": ck.get("sm_mhz"), "reasons": ck.get("reasons")}})
+        del w, acts, ws
+        torch.cuda.empty_cache()
+    return rows
 
 
 # ----------------------------------------------------------------- our arm
@@ -404,10 +530,19 @@ def run_ours(args, rank, world, local_rank):
         "wall_s_timed": wall,
         "e2e": e2e,
     }
+    if not args.no_per_config:
+        del st
+        torch.cuda.empty_cache()
+        line["per_config"] = per_config_rows(dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
-        ms, detail = OracleSample(cfg, seed=0, fp8=args.fp8 or args.attn8).run()
+        ms, detail, measured = OracleSample(cfg, seed=0, fp8=args.fp8 or args.attn8).run()
+        full = oracle_full_block(configs.get("1.3b-short"), cpu_cores())
+        for row in line.get("per_config", []):
+            if row["config"] == full["config"] and row["B"] == 1:
+                full["gpu_block_ms"] = row["block_ms"]
         line["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": cpu_cores(),
-                                "blas_threads": blas_threads(), "kind": "oracle", "sample": detail}
+                                "blas_threads": blas_threads(), "kind": "oracle", "estimated": True,
+                                "measured": measured, "sample": detail, "measured_full_block": full}
     print(json.dumps(line), flush=True)
 
 

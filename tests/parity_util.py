@@ -12,6 +12,36 @@ from video_diffusion_transformer_fwd_b200.configs import BlockConfig
 BF16_REL_L2 = 2e-2      # bf16 configs: relative L2 error bound on sampled rows
 F32_MAX_ABS = 1e-4      # fp32 configs: max-abs error bound
 
+# Canary guard bytes: outputs and workspaces of the parity tests sit inside a
+# larger allocation whose GUARD_BYTES before and after are filled with
+# GUARD_VALUE; a kernel writing past either end of its buffer changes them.
+GUARD_BYTES = 4096      # keeps the buffer's alignment (a multiple of 256)
+GUARD_VALUE = 0xA5
+
+
+class Guarded:
+    """A device tensor of ``shape`` / ``dtype`` (``t``) with canary bytes on
+    both sides; ``check()`` asserts they are untouched."""
+
+    def __init__(self, shape, dtype, device="cuda", init=None):
+        es = torch.empty((), dtype=dtype).element_size()
+        n = 1
+        for d in shape:
+            n *= int(d)
+        self.nbytes = n * es
+        self.raw = torch.full((2 * GUARD_BYTES + self.nbytes,), GUARD_VALUE, dtype=torch.uint8,
+                              device=device)
+        self.t = self.raw[GUARD_BYTES:GUARD_BYTES + self.nbytes].view(dtype).view(*shape)
+        if init is not None:
+            self.t.copy_(init)
+
+    def check(self, what="buffer"):
+        torch.cuda.synchronize()
+        lo = self.raw[:GUARD_BYTES]
+        hi = self.raw[GUARD_BYTES + self.nbytes:]
+        assert bool((lo == GUARD_VALUE).all()), f"{what}: bytes before the buffer overwritten"
+        assert bool((hi == GUARD_VALUE).all()), f"{what}: bytes after the buffer overwritten"
+
 
 def rel_l2(a, b) -> float:
     a = np.asarray(a, np.float64)
@@ -48,13 +78,15 @@ class GpuBlockRun:
             acts["e0"][:, 2] = -self.w["modulation"][2]
             acts["e0"][:, 5] = -self.w["modulation"][5]
         self.x0 = acts["x"].clone()
-        self.x = acts["x"]
+        self._gx = Guarded(tuple(acts["x"].shape), acts["x"].dtype, dev, init=acts["x"])
+        self.x = self._gx.t
         self.ctx = acts["ctx"]
         self.e0 = acts["e0"]
         self.ctx_lens = None if ctx_lens is None else torch.tensor(ctx_lens, dtype=torch.int32,
                                                                     device=dev)
         self.rope = wan.rope_freqs(cfg.head_dim, 1024, cfg.theta, device=dev)
-        self.ws = wan.alloc_workspace(self.dims, B, device=dev)
+        self._gws = Guarded((wan.wan_block_workspace_bytes(self.dims, B),), torch.uint8, dev)
+        self.ws = self._gws.t
 
     def run(self, times=1):
         for _ in range(times):
@@ -62,6 +94,8 @@ class GpuBlockRun:
                               ctx_lens=self.ctx_lens)
         torch.cuda.synchronize()
         assert wan.device_status() == wan.WAN_OK
+        self._gx.check("x")
+        self._gws.check("workspace")
         return self
 
     def ws_rows(self, which, width, rows):

@@ -11,7 +11,7 @@ from oracle import wan_oracle as O
 from video_diffusion_transformer_fwd_b200 import configs, synth, wan
 from video_diffusion_transformer_fwd_b200.configs import BlockConfig
 
-from parity_util import BF16_REL_L2, F32_MAX_ABS, GpuBlockRun, np64, rel_l2, weights64
+from parity_util import BF16_REL_L2, F32_MAX_ABS, GpuBlockRun, Guarded, np64, rel_l2, weights64
 
 pytestmark = pytest.mark.gpu
 
@@ -39,12 +39,14 @@ def test_rope_table(d):
 @pytest.mark.parametrize("cfg", [True, False])
 def test_euler_cfg(vdt, n, cfg):
     g = torch.Generator(device="cuda").manual_seed(7)
-    x = torch.randn(n, device="cuda", generator=g)
+    gx = Guarded((n,), torch.float32, init=torch.randn(n, device="cuda", generator=g))
+    x = gx.t
     vc = torch.randn(n, device="cuda", generator=g).to(synth.TORCH_DTYPES[vdt])
     vu = torch.randn(n, device="cuda", generator=g).to(synth.TORCH_DTYPES[vdt]) if cfg else None
     x0 = np64(x)
     wan.euler_cfg_step(x, vc, vu, 5.0, 0.9, 0.875)
     torch.cuda.synchronize()
+    gx.check("euler x")
     dt = float(np.float32(0.875) - np.float32(0.9))
     ref = O.euler_cfg_step(x0, np64(vc), None if vu is None else np64(vu), 5.0, 0.9, 0.9 + dt)
     assert np.abs(np64(x) - ref).max() <= 1e-5
@@ -61,8 +63,10 @@ def test_euler_cfg_empty():
 def _attn_case(B, Lq, Lk, n, d, dtype, k_lens=None, std=1.0, seed=500):
     q, k, v = synth.attention_inputs(B, Lq, Lk, n, d, dtype, "cuda", seed, std)
     kl = None if k_lens is None else torch.tensor(k_lens, dtype=torch.int32, device="cuda")
-    o = wan.attention(q, k, v, k_lens=kl)
+    go = Guarded(tuple(q.shape), q.dtype)
+    o = wan.attention(q, k, v, k_lens=kl, out=go.t)
     torch.cuda.synchronize()
+    go.check("attention output")
     got = np64(o)
     ref = np.stack([O.attention(np64(q[b]), np64(k[b]), np64(v[b]),
                                 None if k_lens is None else k_lens[b]) for b in range(B)])
