@@ -60,6 +60,9 @@ def parse_args():
                     help="FP8 GEMM mode of the blocks (e4m3 projections, bf16 attention); not the default")
     ap.add_argument("--attn8", action="store_true",
                     help="FP8 GEMMs and the 8-bit self-attention (int8 Q K^T, e4m3 P V); not the default")
+    ap.add_argument("--ulysses", action="store_true",
+                    help="all ranks form one sequence-parallel group: tokens sharded, every block's self-attention "
+                         "head-parallel between two all-to-alls (strong scaling); not the default")
     ap.add_argument("--cfg-parallel", action="store_true",
                     help="ranks 2p / 2p+1 run the conditional / unconditional branch of one step and "
                          "exchange their block outputs (even --gpus); not the default")
@@ -316,15 +319,17 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(cfg, world, cfg_parallel=False):
+def workload_config(cfg, world, cfg_parallel=False, ulysses=False):
     return {
         "workload": (f"{cfg.name}: {cfg.blocks} WanAttentionBlocks dim {cfg.dim}, {cfg.heads} heads "
                      f"(head_dim {cfg.head_dim}), ffn {cfg.ffn_dim}, grid {cfg.F}x{cfg.H}x{cfg.W} "
                      f"(L={cfg.L}), text {cfg.text_len}, cond+uncond batched (B=2), CFG "
                      f"{cfg.guide_scale}, Euler sigma {cfg.sigma}->{cfg.sigma_next}"),
         "seq_len": cfg.L, "batch_per_gpu": 1 if cfg_parallel else 2, "blocks": cfg.blocks,
-        "global_batch": world if cfg_parallel else 2 * world,
-        "parallelism": ("cfg-pairs (branch outputs all-gathered within each pair)" if cfg_parallel else
+        "global_batch": 2 if ulysses else world if cfg_parallel else 2 * world,
+        "parallelism": (f"ulysses-{world} (tokens sharded, self-attention head-parallel between two "
+                        f"all-to-alls per block)" if ulysses else
+                        "cfg-pairs (branch outputs all-gathered within each pair)" if cfg_parallel else
                         "replicas" if world > 1 else "single"),
         "l2": "inputs larger than L2 (28 GB of block weights and a 671 MB token state per step)",
         "weights": "random N(0,0.02), synthetic x/ctx N(0,1)",
@@ -395,12 +400,17 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     from video_diffusion_transformer_fwd_b200 import configs, wan
-    from video_diffusion_transformer_fwd_b200.step import CFGParallelStep, DenoiseStep, cfg_pairs
+    from video_diffusion_transformer_fwd_b200.step import CFGParallelStep, DenoiseStep, UlyssesStep, cfg_pairs
 
     torch.cuda.set_device(local_rank)
     dev = f"cuda:{local_rank}"
     cfg = configs.get(args.config)
-    if args.cfg_parallel:
+    if args.ulysses:
+        if args.fp8 or args.attn8 or args.cfg_parallel:
+            raise SystemExit("--ulysses runs the bf16 blocks on the batched CFG pair")
+        st = UlyssesStep(cfg, rank, world, group=dist.group.WORLD if world > 1 else None, seed=0, device=dev,
+                         exchange=None if world > 1 else (lambda send, recv, group: recv.copy_(send)))
+    elif args.cfg_parallel:
         if args.fp8 or args.attn8:
             raise SystemExit("--cfg-parallel runs the bf16 blocks")
         groups = [dist.new_group(pr) for pr in cfg_pairs(world)]     # every rank creates every group
@@ -408,6 +418,10 @@ def run_ours(args, rank, world, local_rank):
     else:
         st = DenoiseStep(cfg, seed=1000 * rank, device=dev, fp8=args.fp8, attn8=args.attn8)
     seqs = 1 if args.cfg_parallel else 2          # sequences of the CFG pair each rank runs
+    # CFG pairs the job completes per step: one per rank (replicas), one per
+    # rank pair (CFG-parallel), one for the whole group (Ulysses)
+    pairs = 1 if args.ulysses else world * seqs // 2
+    shards = world if args.ulysses else 1
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -469,21 +483,24 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         e_ms = max_over_ranks(e_start.elapsed_time(e_end), world, dev)
-        e2e = {"value": per_block_ms(e_ms, args.steps, cfg.blocks, world * seqs // 2), "unit": UNIT,
+        e2e = {"value": per_block_ms(e_ms, args.steps, cfg.blocks, pairs), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     if rank != 0:
         return
-    value = per_block_ms(ms_max, args.steps, cfg.blocks, world * seqs // 2)
+    value = per_block_ms(ms_max, args.steps, cfg.blocks, pairs)
     peaks, peak_src = read_peaks()
     blocks_run = args.steps * cfg.blocks
     import dataclasses
     c2 = dataclasses.replace(cfg, batch=seqs)
     attn_n, attn_ms = prof["attn_self"]
     gemm_n, gemm_ms = prof["gemm_tc"]
-    attn_flops_launch = c2.self_attn_flops()
+    attn_flops_launch = c2.self_attn_flops() / shards          # this rank's heads
+    # this rank's GEMM work: its token rows, and the replicated cross K/V projection
+    gemm_flops_block = (c2.gemm_flops() - seqs * 4.0 * cfg.text_len * cfg.dim * cfg.dim) / shards \
+        + seqs * 4.0 * cfg.text_len * cfg.dim * cfg.dim
     attn_tflops = attn_flops_launch * attn_n / (attn_ms * 1e-3) / 1e12 if attn_ms > 0 else None
-    gemm_tflops = c2.gemm_flops() * blocks_run / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
+    gemm_tflops = gemm_flops_block * blocks_run / (gemm_ms * 1e-3) / 1e12 if gemm_ms > 0 else None
     # dominant kernel class by device time
     dom = max(prof.items(), key=lambda kv: kv[1][1])[0]
     peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
@@ -492,11 +509,11 @@ def run_ours(args, rank, world, local_rank):
         avg_ms = attn_ms / attn_n
         tr = TRAFFIC.get("attn_self")
         traffic = None
-        if tr and not args.attn8 and tr.get("source_sha") == source_hash(*ATTN_SOURCES):
+        if tr and not args.attn8 and shards == 1 and tr.get("source_sha") == source_hash(*ATTN_SOURCES):
             traffic = tr["bytes_per_launch"] * seqs / 2     # recorded for the B = 2 launch
         apk = peak_sust * (2.0 if args.attn8 else 1.0)
         roofline = {"kernel": ("attn8 (8-bit self-attention incl. its quantization passes" if args.attn8 else
-                               "attn_tc (self-attention") + f", B={seqs}, L=32760, 40 heads, d=128)",
+                               "attn_tc (self-attention") + f", B={seqs}, L={cfg.L}, {cfg.heads // shards} heads, d=128)",
                     "bound": "tensor", "achieved": attn_flops_launch / (avg_ms * 1e-3) / 1e12,
                     "peak": apk, "unit": "TFLOP/s",
                     "frac": attn_flops_launch / (avg_ms * 1e-3) / 1e12 / apk,
@@ -513,12 +530,12 @@ def run_ours(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None,
+        "scaling": "strong" if args.ulysses else "weak", "vs_baseline": None,
         "dtype": ("fp8 e4m3 GEMMs, int8 QK^T / e4m3 PV self-attention" if args.attn8 else
                   "fp8 e4m3 GEMMs (per-token / per-tensor scales), bf16 attention" if args.fp8 else "bf16"),
         "data": "synthetic",
         "impl": "ours",
-        "config": workload_config(cfg, world, args.cfg_parallel),
+        "config": workload_config(cfg, world, args.cfg_parallel, args.ulysses),
         "attention_tflops": attn_tflops, "gemm_tflops": gemm_tflops,
         "attention_frac_of_2250": None if attn_tflops is None else attn_tflops / 2250.0,
         "gemm_frac_of_2250": None if gemm_tflops is None else gemm_tflops / 2250.0,

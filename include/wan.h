@@ -210,6 +210,71 @@ int wan_block_forward_noalloc(const wan_dims *dims, int B, float *x, const void 
                               int rope_max_pos, wan_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Sequence-parallel (head-parallel, "Ulysses") phases of the block
+ * ([DIGEST] training/inference-system section, 2D context parallelism:
+ * Ulysses inside Ring; [WALK] CLI, --ulysses). N ranks each hold a token
+ * shard of the sequence; around the self-attention an all-to-all gives every
+ * rank all tokens of n/N heads and a second one returns the outputs:
+ *   wan_block_sp_qkv     LN1 + modulate, QKV projection, q / k RMSNorm and
+ *                        3D RoPE on the rank's rows -> q | k | v per row
+ *   (caller) all-to-all  token shards -> head shards (wan_permute_chunks
+ *                        packs and unpacks the exchanged buffers)
+ *   wan_attention        all tokens, the rank's n/N heads
+ *   (caller) all-to-all  head shards -> token shards
+ *   wan_block_sp_finish  output projection + gated residual, cross-attention
+ *                        branch, FFN branch on the rank's rows
+ * With N = 1 (one shard = the whole sequence) the phases compute the block of
+ * wan_block_forward; bf16 differs only in rounding q after its RMS factor
+ * (wan_block_forward applies that factor inside the attention). WAN_F32 and
+ * WAN_BF16 only.
+ * ------------------------------------------------------------------------- */
+
+/* Workspace bytes of wan_block_sp_qkv / wan_block_sp_finish for B sequences
+ * of `rows` token rows each (0 on invalid arguments). */
+size_t wan_block_sp_workspace_bytes(const wan_dims *dims, int B, int rows);
+
+/* wan_block_sp_qkv -- the self-attention inputs of a token shard.
+ *   dims      the whole problem (grid (F, H, W) gives the RoPE positions).
+ *   rows      tokens of each sequence held here; row r is token tok0 + r of
+ *             the grid (tok0 + rows <= F*H*W).
+ *   x         float32 [B, rows, dim]; e0 as in wan_block_forward (per token:
+ *             [B, rows, 6, dim], the shard's rows).
+ *   qkv       out, (dt) [B, rows, 3*dim]: q | k | v of each row; q and k
+ *             RMS-normalised with their gains and rotated by the 3D RoPE.
+ *   workspace ws_bytes >= wan_block_sp_workspace_bytes(dims, B, rows).
+ * Errors as wan_block_forward; WAN_EINVAL for a shard outside the grid,
+ * WAN_EUNSUPPORTED for WAN_FP8 modes. */
+int wan_block_sp_qkv(const wan_dims *dims, int B, int rows, int tok0, const float *x,
+                     const float *e0, const wan_block_weights *w, const float *rope,
+                     int rope_max_pos, void *qkv, void *workspace, size_t ws_bytes,
+                     wan_stream_t stream);
+
+/* wan_block_sp_finish -- the rest of the block on a token shard:
+ *   x += m2 * (o W_o^T + b_o); x += CrossAttn(norm3 x, ctx); x += m5 * FFN(...)
+ *   x         in/out float32 [B, rows, dim] (the shard's rows).
+ *   ctx, ctx_lens, e0, w  as in wan_block_forward (e0 per token: the shard's rows).
+ *   o         (dt) [B, rows, dim] self-attention output of the shard's rows,
+ *             all heads (heads in order within a row).
+ * Errors as wan_block_sp_qkv. */
+int wan_block_sp_finish(const wan_dims *dims, int B, int rows, float *x, const void *ctx,
+                        const int *ctx_lens, const float *e0, const wan_block_weights *w,
+                        const void *o, void *workspace, size_t ws_bytes, wan_stream_t stream);
+
+/* wan_permute_chunks -- dst = src with its axes permuted, in units of
+ * chunk_bytes: src is row-major [dims[0]]...[dims[ndim-1]] chunks, dst is
+ * row-major over axes perm[0], ..., perm[ndim-1] of src (dst axis k runs over
+ * src axis perm[k]). Used to pack and unpack the all-to-all buffers of the
+ * sequence-parallel attention, e.g. q|k|v rows [B][rows][3][N][n/N*d] ->
+ * per-destination [N][B][rows][3][n/N*d] with perm (3, 0, 1, 2).
+ *   ndim 1..5; chunk_bytes a positive multiple of 16; src and dst device
+ *   buffers of prod(dims) * chunk_bytes bytes each, 16-byte aligned, not
+ *   overlapping.
+ * Errors: WAN_EINVAL (bad ndim / perm / chunk size, overlap, NULL),
+ * WAN_EALIGN. */
+int wan_permute_chunks(const void *src, void *dst, int ndim, const int *dims,
+                       const int *perm, size_t chunk_bytes, wan_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Whole-model forward on latents ([WALK] WanModel structure and forward
  * snippets, time-projection snippet; [DIFFUSERS] "3D Patchify", "Unpatchify").
  *   x   = Conv3d(C_in, dim, kernel = stride = (1,2,2))(latent), flattened to

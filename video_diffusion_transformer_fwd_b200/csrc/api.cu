@@ -118,6 +118,8 @@ static int check_dims(const wan_dims *d, int B) {
     return set_error(WAN_EUNSUPPORTED, "dtype %d", d->dtype);
   const int hd = d->dim / d->heads;
   if (d->dtype != WAN_F32 && hd != 128) return set_error(WAN_EUNSUPPORTED, "bf16 / fp8 paths need head_dim 128 (got %d)", hd);
+  if (d->dtype != WAN_F32 && B > 65535)
+    return set_error(WAN_EUNSUPPORTED, "bf16 / fp8 paths take at most 65535 sequences a call (got %d)", B);
   if (d->dtype != WAN_F32 && d->dim % 256)
     return set_error(WAN_EUNSUPPORTED, "bf16 / fp8 paths need dim %% 256 == 0 (got %d): the QKV epilogue "
                                        "normalises q and k over whole 256-column tiles", d->dim);
@@ -131,10 +133,12 @@ static int check_dims(const wan_dims *d, int B) {
   return WAN_OK;
 }
 
-static WsLayout layout_of(const wan_dims *d, int B) {
+// Workspace of a block call on `rows` token rows per sequence (the whole
+// sequence, or one rank's shard in the sequence-parallel phases).
+static WsLayout layout_rows(const wan_dims *d, int B, int rows) {
   WsLayout w;
   const size_t es = dtype_size(d->dtype);
-  const size_t BL = (size_t)B * d->F * d->H * d->W, D = d->dim, T = d->text_len, Fh = d->ffn_dim;
+  const size_t BL = (size_t)B * rows, D = d->dim, T = d->text_len, Fh = d->ffn_dim;
   const size_t sz[WAN_WS_COUNT] = {
       BL * D * es,            // ACT
       BL * 3 * D * es,        // QKV
@@ -147,7 +151,7 @@ static WsLayout layout_of(const wan_dims *d, int B) {
       (BL > (size_t)B * T ? BL : (size_t)B * T) * 4 * (D >= 256 ? D / 256 : 1) * 4,   // STATS: per-row partial sums of squares
       is_fp8(d->dtype) ? (BL * Fh > (size_t)B * T * D ? BL * Fh : (size_t)B * T * D) : 0,   // A8
       is_fp8(d->dtype) ? (BL > (size_t)B * T ? BL : (size_t)B * T) * 4 : 0,                // ASCALE
-      d->dtype == WAN_FP8_ATTN && B > 0 ? attention_8bit_ws_bytes(B, d->heads, d->F * d->H * d->W, d->F * d->H * d->W) : 0,
+      d->dtype == WAN_FP8_ATTN && B > 0 ? attention_8bit_ws_bytes(B, d->heads, rows, rows) : 0,
   };
   size_t o = 0;
   for (int i = 0; i < WAN_WS_COUNT; ++i) {
@@ -157,6 +161,7 @@ static WsLayout layout_of(const wan_dims *d, int B) {
   w.total = o;
   return w;
 }
+static WsLayout layout_of(const wan_dims *d, int B) { return layout_rows(d, B, d->F * d->H * d->W); }
 
 // ---------------------------------------------------------------- FP8 block
 // The fused bf16 block with every projection on the FP8 tensor cores
@@ -290,6 +295,243 @@ static int block_forward_fp8(const wan_dims &d, int B, float *x, const void *ctx
   return WAN_OK;
 }
 
+// ---------------------------------------------------------------- block stages
+// One block call on `rows` token rows of each of B sequences; row r of a
+// sequence is token tok0 + r of its (F, H, W) grid. wan_block_forward runs the
+// stages on whole sequences; the sequence-parallel entry points run the first
+// and the last on one rank's token shard, the attention between them running
+// on a head shard of the whole sequence after an all-to-all.
+struct BlockCall {
+  const wan_dims *d;
+  int B, rows, tok0;
+  float *x;
+  const void *ctx;
+  const int *ctx_lens;
+  const float *e0;
+  const wan_block_weights *w;
+  const float *rope;
+  int rope_max_pos;
+  char *ws;
+  WsLayout lay;
+  cudaStream_t s;
+  ModSrc ms;
+};
+
+static int parts_of(int D) { return D >= 256 ? D / 256 : 1; }
+
+// m = modulation + e0 (shift, scale, gate, shift2, scale2, gate2) into the
+// workspace, unless e0 is per token (then read in place)
+static int stage_mod(const BlockCall &c) {
+  if (c.ms.ptok) return WAN_OK;
+  return WAN_PROF(WAN_K_MISC, c.s, launch_mod_combine(c.w->modulation, c.e0, const_cast<float *>(c.ms.mod),
+                                                      c.B, c.d->dim, c.s));
+}
+
+// LN1 + modulate, the QKV projection, q / k RMSNorm and 3D RoPE into qkv
+// [B * rows, 3 * dim] (q | k | v per row). bf16: the GEMM epilogue leaves
+// the rows' sums of squares in the workspace statistics; k is scaled by its
+// RMS factor here, q too when `normalize_q` (otherwise the attention folds
+// q's factor into its logit scale).
+static int stage_self_qkv(const BlockCall &c, void *qkv, bool normalize_q) {
+  const wan_dims &d = *c.d;
+  const int D = d.dim, hd = D / d.heads, BL = c.B * c.rows, dt = d.dtype;
+  const size_t es = dtype_size(dt);
+  void *act = c.ws + c.lay.off[WAN_WS_ACT];
+  float *stats = reinterpret_cast<float *>(c.ws + c.lay.off[WAN_WS_STATS]);
+  const int parts = parts_of(D), sstride = 4 * parts;
+  int rc;
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, c.s, launch_layernorm_mod(c.x, act, dt, BL, D, ln_of(c.ms, 0, 1), nullptr,
+                                                                nullptr, d.eps, c.s)))) return rc;
+  GemmArgs g = {};
+  g.M = BL; g.N = 3 * D; g.K = D; g.A = act; g.lda = D;
+  g.Bseg[0] = c.w->wq; g.Bseg[1] = c.w->wk; g.Bseg[2] = c.w->wv;
+  g.bias[0] = c.w->bq; g.bias[1] = c.w->bk; g.bias[2] = c.w->bv;
+  g.segN = D; g.nseg = 3; g.C = qkv; g.ldc = 3 * D;
+  g.rope = c.rope; g.F = d.F; g.H = d.H; g.W = d.W; g.head_dim = hd; g.rows_per_seq = c.rows; g.tok0 = c.tok0;
+  char *q = static_cast<char *>(qkv);
+  if (dt == WAN_BF16) {
+    g.epi = EPI_QKNORM;
+    g.gamma[0] = c.w->gq; g.gamma[1] = c.w->gk; g.gamma[2] = nullptr;
+    g.ss = stats; g.ss_stride = sstride; g.ss_col[0] = 0; g.ss_col[1] = 1; g.ss_col[2] = -1;
+    g.rope_mask = 3;
+    if ((rc = run_gemm(g, dt, c.s))) return rc;
+    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, c.s, launch_scale_rows(q + D * es, BL, 3 * D, D, stats + parts, sstride,
+                                                                 parts, d.eps, c.s)))) return rc;
+    if (normalize_q &&
+        (rc = WAN_PROF(WAN_K_QKNORM_ROPE, c.s, launch_scale_rows(q, BL, 3 * D, D, stats, sstride, parts, d.eps, c.s))))
+      return rc;
+    return WAN_OK;
+  }
+  g.epi = EPI_STORE;
+  if ((rc = run_gemm(g, dt, c.s))) return rc;
+  if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, c.s, launch_rmsnorm_rope(q, dt, BL, 3 * D, D, hd, c.w->gq, d.eps, c.rope,
+                                                                 c.rope_max_pos, d.F, d.H, d.W, c.s, c.rows,
+                                                                 c.tok0)))) return rc;
+  return WAN_PROF(WAN_K_QKNORM_ROPE, c.s, launch_rmsnorm_rope(q + D * es, dt, BL, 3 * D, D, hd, c.w->gk, d.eps, c.rope,
+                                                              c.rope_max_pos, d.F, d.H, d.W, c.s, c.rows, c.tok0));
+}
+
+// Self-attention of whole sequences (rows == L) from the stage_self_qkv
+// output; bf16 folds q's RMS factor into the logit scale.
+static int stage_self_attention(const BlockCall &c, const void *qkv, void *o) {
+  const wan_dims &d = *c.d;
+  const int D = d.dim, hd = D / d.heads;
+  const size_t es = dtype_size(d.dtype);
+  const char *q = static_cast<const char *>(qkv);
+  AttnArgs a = {};
+  a.B = c.B; a.heads = d.heads; a.Lq = c.rows; a.Lk = c.rows; a.d = hd;
+  a.q = q; a.ldq = 3 * D; a.k = q + D * es; a.ldk = 3 * D; a.v = q + 2 * D * es; a.ldv = 3 * D;
+  a.o = o; a.ldo = D; a.k_lens = nullptr; a.scale = 1.0f / sqrtf((float)hd);
+  if (d.dtype == WAN_BF16) {
+    const int parts = parts_of(D);
+    a.q_ss = reinterpret_cast<const float *>(c.ws + c.lay.off[WAN_WS_STATS]); a.q_ss_stride = 4 * parts;
+    a.q_ss_parts = parts; a.q_ss_n = (float)D; a.q_ss_eps = d.eps;
+  }
+  return run_attention(a, d.dtype, c.s, WAN_K_ATTN_SELF);
+}
+
+// The rest of the block on the call's rows: x += m2 * (o W_o^T + b_o), the
+// cross-attention branch (ungated) and the FFN branch.
+static int stage_finish(const BlockCall &c, const void *o) {
+  const wan_dims &d = *c.d;
+  const int D = d.dim, T = d.text_len, Fh = d.ffn_dim, hd = D / d.heads, BL = c.B * c.rows, dt = d.dtype;
+  const size_t es = dtype_size(dt);
+  const bool tc = dt == WAN_BF16;
+  void *act = c.ws + c.lay.off[WAN_WS_ACT];
+  void *qc = c.ws + c.lay.off[WAN_WS_QC];
+  char *kvc = c.ws + c.lay.off[WAN_WS_KVC];
+  void *oc = c.ws + c.lay.off[WAN_WS_OC];
+  void *hbuf = c.ws + c.lay.off[WAN_WS_H];
+  float *stats = reinterpret_cast<float *>(c.ws + c.lay.off[WAN_WS_STATS]);
+  const int parts = parts_of(D), sstride = 4 * parts;
+  int rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = D; g.A = o; g.lda = D;
+    g.Bseg[0] = c.w->wo; g.bias[0] = c.w->bo; g.segN = D; g.nseg = 1;
+    g.epi = EPI_RESID; g.X = c.x; g.ldx = D;
+    gate_of(c.ms, g, 2);
+    if ((rc = run_gemm(g, dt, c.s))) return rc;
+  }
+
+  // ---- cross-attention branch (ungated): x += Wco . Attn(q(norm3 x), k(ctx), v(ctx))
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, c.s, launch_layernorm_mod(c.x, act, dt, BL, D, LnMod{}, c.w->g3, c.w->b3,
+                                                                d.eps, c.s)))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = D; g.A = act; g.lda = D;
+    g.Bseg[0] = c.w->cwq; g.bias[0] = c.w->cbq; g.segN = D; g.nseg = 1;
+    g.C = qc; g.ldc = D;
+    g.epi = tc ? EPI_QKNORM : EPI_STORE;
+    g.gamma[0] = c.w->cgq; g.ss = stats; g.ss_stride = sstride; g.ss_col[0] = 2; g.ss_col[1] = g.ss_col[2] = -1;
+    if ((rc = run_gemm(g, dt, c.s))) return rc;
+  }
+  if (!tc && (rc = WAN_PROF(WAN_K_QKNORM_ROPE, c.s, launch_rmsnorm_rope(qc, dt, BL, D, D, hd, c.w->cgq, d.eps, nullptr,
+                                                                        0, 1, 1, 1, c.s)))) return rc;
+  if (T > 0) {
+    GemmArgs g = {};
+    g.M = c.B * T; g.N = 2 * D; g.K = D; g.A = c.ctx; g.lda = D;
+    g.Bseg[0] = c.w->cwk; g.Bseg[1] = c.w->cwv; g.bias[0] = c.w->cbk; g.bias[1] = c.w->cbv;
+    g.segN = D; g.nseg = 2; g.C = kvc; g.ldc = 2 * D;
+    g.epi = tc ? EPI_QKNORM : EPI_STORE;
+    g.gamma[0] = c.w->cgk; g.gamma[1] = nullptr; g.ss = stats; g.ss_stride = sstride;
+    g.ss_col[0] = 3; g.ss_col[1] = -1; g.ss_col[2] = -1;
+    if ((rc = run_gemm(g, dt, c.s))) return rc;
+    if (tc) {
+      if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, c.s, launch_scale_rows(kvc, c.B * T, 2 * D, D, stats + 3 * parts, sstride,
+                                                                   parts, d.eps, c.s)))) return rc;
+    } else if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, c.s, launch_rmsnorm_rope(kvc, dt, c.B * T, 2 * D, D, hd, c.w->cgk,
+                                                                          d.eps, nullptr, 0, 1, 1, 1, c.s)))) {
+      return rc;
+    }
+  }
+  {
+    AttnArgs a = {};
+    a.B = c.B; a.heads = d.heads; a.Lq = c.rows; a.Lk = T; a.d = hd;
+    a.q = qc; a.ldq = D; a.k = kvc; a.ldk = 2 * D; a.v = kvc + D * es; a.ldv = 2 * D;
+    a.o = oc; a.ldo = D; a.k_lens = c.ctx_lens; a.scale = 1.0f / sqrtf((float)hd);
+    if (tc) {
+      a.q_ss = stats + 2 * parts; a.q_ss_stride = sstride; a.q_ss_parts = parts;
+      a.q_ss_n = (float)D; a.q_ss_eps = d.eps;
+    }
+    if ((rc = run_attention(a, dt, c.s, WAN_K_ATTN_CROSS))) return rc;
+  }
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = D; g.A = oc; g.lda = D;
+    g.Bseg[0] = c.w->cwo; g.bias[0] = c.w->cbo; g.segN = D; g.nseg = 1;
+    g.epi = EPI_RESID; g.X = c.x; g.ldx = D; g.gate = nullptr; g.rows_per_gate = c.rows;
+    if ((rc = run_gemm(g, dt, c.s))) return rc;
+  }
+
+  // ---- FFN branch: x += m5 * W2 . gelu_tanh(W1 . (LN(x)(1 + m4) + m3))
+  if ((rc = WAN_PROF(WAN_K_LAYERNORM, c.s, launch_layernorm_mod(c.x, act, dt, BL, D, ln_of(c.ms, 3, 4), nullptr,
+                                                                nullptr, d.eps, c.s)))) return rc;
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = Fh; g.K = D; g.A = act; g.lda = D;
+    g.Bseg[0] = c.w->w1; g.bias[0] = c.w->b1; g.segN = Fh; g.nseg = 1;
+    g.epi = EPI_GELU; g.C = hbuf; g.ldc = Fh;
+    if ((rc = run_gemm(g, dt, c.s))) return rc;
+  }
+  {
+    GemmArgs g = {};
+    g.M = BL; g.N = D; g.K = Fh; g.A = hbuf; g.lda = Fh;
+    g.Bseg[0] = c.w->w2; g.bias[0] = c.w->b2; g.segN = D; g.nseg = 1;
+    g.epi = EPI_RESID; g.X = c.x; g.ldx = D;
+    gate_of(c.ms, g, 5);
+    if ((rc = run_gemm(g, dt, c.s))) return rc;
+  }
+  return WAN_OK;
+}
+
+// Checks shared by the block entry points; fills the call on success.
+// `need_ctx` / `need_rope`: the call runs the cross-attention / the RoPE.
+static int prepare_call(BlockCall &c, const wan_dims *dims, int B, int rows, int tok0, float *x, const void *ctx,
+                        const int *ctx_lens, const float *e0, const wan_block_weights *w, const float *rope,
+                        int rope_max_pos, void *workspace, size_t ws_bytes, cudaStream_t s, bool need_ctx,
+                        bool need_rope) {
+  const wan_dims &d = *dims;
+  if (!w) return set_error(WAN_EINVAL, "weights is NULL");
+  const void *ptrs[] = {x, e0, workspace, w->modulation, w->wq, w->bq, w->wk, w->bk, w->wv,
+                        w->bv, w->wo, w->bo, w->gq, w->gk, w->g3, w->b3, w->cwq, w->cbq, w->cwk,
+                        w->cbk, w->cwv, w->cbv, w->cwo, w->cbo, w->cgq, w->cgk, w->w1, w->b1,
+                        w->w2, w->b2, need_rope ? rope : x};
+  for (size_t i = 0; i < sizeof(ptrs) / sizeof(ptrs[0]); ++i) {
+    if (!ptrs[i]) return set_error(WAN_EINVAL, "pointer argument #%zu is NULL", i);
+    if (!aligned16(ptrs[i])) return set_error(WAN_EALIGN, "pointer argument #%zu not 16-byte aligned", i);
+  }
+  if (is_fp8(d.dtype)) {
+    if (!w->w_scales) return set_error(WAN_EINVAL, "WAN_FP8 needs w_scales");
+    if (!aligned16(w->w_scales)) return set_error(WAN_EALIGN, "w_scales not 16-byte aligned");
+  }
+  if (need_ctx && d.text_len > 0 && !ctx) return set_error(WAN_EINVAL, "ctx is NULL");
+  if (ctx && !aligned16(ctx)) return set_error(WAN_EALIGN, "ctx not 16-byte aligned");
+  if (ctx_lens && !aligned16(ctx_lens)) return set_error(WAN_EALIGN, "ctx_lens not 16-byte aligned");
+  if (need_rope) {
+    const int gmax = d.F > d.H ? (d.F > d.W ? d.F : d.W) : (d.H > d.W ? d.H : d.W);
+    if (rope_max_pos < gmax) return set_error(WAN_EINVAL, "rope table has %d rows, grid needs %d", rope_max_pos, gmax);
+  }
+  c.lay = layout_rows(dims, B, rows);
+  if (ws_bytes < c.lay.total) return set_error(WAN_EINVAL, "workspace %zu bytes < %zu needed", ws_bytes, c.lay.total);
+  c.d = dims; c.B = B; c.rows = rows; c.tok0 = tok0; c.x = x; c.ctx = ctx; c.ctx_lens = ctx_lens; c.e0 = e0;
+  c.w = w; c.rope = rope; c.rope_max_pos = rope_max_pos; c.ws = static_cast<char *>(workspace); c.s = s;
+  c.ms = ModSrc{d.e0_per_token != 0, e0, reinterpret_cast<float *>(c.ws + c.lay.off[WAN_WS_MOD]), w->modulation,
+                rows, d.dim};
+  return WAN_OK;
+}
+
+// Rows and first token of a sequence-parallel call, and its dtype.
+static int check_shard(const wan_dims *dims, int B, int rows, int tok0) {
+  int rc = check_dims(dims, B);
+  if (rc) return rc;
+  const long long L = (long long)dims->F * dims->H * dims->W;
+  if (rows < 1 || tok0 < 0 || tok0 + (long long)rows > L)
+    return set_error(WAN_EINVAL, "token shard [%d, %d + %d) outside the %lld-token grid", tok0, tok0, rows, L);
+  if (is_fp8(dims->dtype)) return set_error(WAN_EUNSUPPORTED, "the sequence-parallel phases run WAN_F32 or WAN_BF16");
+  return WAN_OK;
+}
+
 }  // namespace wan
 
 using namespace wan;
@@ -325,160 +567,78 @@ int wan_block_forward(const wan_dims *dims, int B, float *x, const void *ctx, co
   int rc = check_dims(dims, B);
   if (rc) return rc;
   if (B == 0) return WAN_OK;
-  if (!w) return set_error(WAN_EINVAL, "weights is NULL");
   const wan_dims &d = *dims;
-  const int L = d.F * d.H * d.W, D = d.dim, T = d.text_len, Fh = d.ffn_dim, hd = D / d.heads;
-  const int dt = d.dtype;
-  const size_t es = dtype_size(dt);
+  const int L = d.F * d.H * d.W;
+  BlockCall c;
+  if ((rc = prepare_call(c, dims, B, L, 0, x, ctx, ctx_lens, e0, w, rope, rope_max_pos, workspace, ws_bytes,
+                         (cudaStream_t)stream, true, true))) return rc;
+  if ((rc = stage_mod(c))) return rc;
+  if (is_fp8(d.dtype)) return block_forward_fp8(d, B, x, ctx, ctx_lens, w, rope, c.ws, c.lay, c.ms, c.s);
+  void *qkv = c.ws + c.lay.off[WAN_WS_QKV];
+  void *o = c.ws + c.lay.off[WAN_WS_O];
+  if ((rc = stage_self_qkv(c, qkv, false))) return rc;
+  if ((rc = stage_self_attention(c, qkv, o))) return rc;
+  return stage_finish(c, o);
+}
+
+size_t wan_block_sp_workspace_bytes(const wan_dims *dims, int B, int rows) {
+  if (check_shard(dims, B, rows, 0) != WAN_OK) return 0;
+  return layout_rows(dims, B, rows).total;
+}
+
+int wan_block_sp_qkv(const wan_dims *dims, int B, int rows, int tok0, const float *x, const float *e0,
+                     const wan_block_weights *w, const float *rope, int rope_max_pos, void *qkv,
+                     void *workspace, size_t ws_bytes, wan_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_shard(dims, B, rows, tok0);
+  if (rc) return rc;
+  if (B == 0) return WAN_OK;
+  if (!qkv) return set_error(WAN_EINVAL, "qkv is NULL");
+  if (!aligned16(qkv)) return set_error(WAN_EALIGN, "qkv not 16-byte aligned");
+  BlockCall c;
+  if ((rc = prepare_call(c, dims, B, rows, tok0, const_cast<float *>(x), nullptr, nullptr, e0, w, rope,
+                         rope_max_pos, workspace, ws_bytes, (cudaStream_t)stream, false, true))) return rc;
+  if ((rc = stage_mod(c))) return rc;
+  return stage_self_qkv(c, qkv, true);
+}
+
+int wan_block_sp_finish(const wan_dims *dims, int B, int rows, float *x, const void *ctx, const int *ctx_lens,
+                        const float *e0, const wan_block_weights *w, const void *o, void *workspace,
+                        size_t ws_bytes, wan_stream_t stream) {
+  g_msg[0] = 0;
+  int rc = check_shard(dims, B, rows, 0);
+  if (rc) return rc;
+  if (B == 0) return WAN_OK;
+  if (!o) return set_error(WAN_EINVAL, "o is NULL");
+  if (!aligned16(o)) return set_error(WAN_EALIGN, "o not 16-byte aligned");
+  BlockCall c;
+  if ((rc = prepare_call(c, dims, B, rows, 0, x, ctx, ctx_lens, e0, w, nullptr, 0, workspace, ws_bytes,
+                         (cudaStream_t)stream, true, false))) return rc;
+  if ((rc = stage_mod(c))) return rc;
+  return stage_finish(c, o);
+}
+
+int wan_permute_chunks(const void *src, void *dst, int ndim, const int *dims, const int *perm, size_t chunk_bytes,
+                       wan_stream_t stream) {
+  g_msg[0] = 0;
+  if (ndim < 1 || ndim > 5 || !dims || !perm) return set_error(WAN_EINVAL, "ndim %d must be 1..5 with dims and perm", ndim);
+  if (chunk_bytes == 0 || chunk_bytes % 16) return set_error(WAN_EINVAL, "chunk_bytes %zu must be a positive multiple of 16", chunk_bytes);
+  bool seen[5] = {false, false, false, false, false};
+  long long n = 1;
+  for (int k = 0; k < ndim; ++k) {
+    if (dims[k] < 0) return set_error(WAN_EINVAL, "dims[%d] = %d < 0", k, dims[k]);
+    if (perm[k] < 0 || perm[k] >= ndim || seen[perm[k]]) return set_error(WAN_EINVAL, "perm is not a permutation");
+    seen[perm[k]] = true;
+    n *= dims[k];
+  }
+  if (n == 0) return WAN_OK;
+  if (!src || !dst) return set_error(WAN_EINVAL, "NULL buffer");
+  if (!aligned16(src) || !aligned16(dst)) return set_error(WAN_EALIGN, "buffers must be 16-byte aligned");
+  const size_t bytes = (size_t)n * chunk_bytes;
+  const char *a = static_cast<const char *>(src), *b = static_cast<const char *>(dst);
+  if (a < b + bytes && b < a + bytes) return set_error(WAN_EINVAL, "src and dst overlap");
   cudaStream_t s = (cudaStream_t)stream;
-
-  const void *ptrs[] = {x, e0, rope, workspace, w->modulation, w->wq, w->bq, w->wk, w->bk, w->wv,
-                        w->bv, w->wo, w->bo, w->gq, w->gk, w->g3, w->b3, w->cwq, w->cbq, w->cwk,
-                        w->cbk, w->cwv, w->cbv, w->cwo, w->cbo, w->cgq, w->cgk, w->w1, w->b1,
-                        w->w2, w->b2};
-  for (size_t i = 0; i < sizeof(ptrs) / sizeof(ptrs[0]); ++i) {
-    if (!ptrs[i]) return set_error(WAN_EINVAL, "pointer argument #%zu is NULL", i);
-    if (!aligned16(ptrs[i])) return set_error(WAN_EALIGN, "pointer argument #%zu not 16-byte aligned", i);
-  }
-  if (is_fp8(dt)) {
-    if (!w->w_scales) return set_error(WAN_EINVAL, "WAN_FP8 needs w_scales");
-    if (!aligned16(w->w_scales)) return set_error(WAN_EALIGN, "w_scales not 16-byte aligned");
-  }
-  if (T > 0 && !ctx) return set_error(WAN_EINVAL, "ctx is NULL");
-  if (ctx && !aligned16(ctx)) return set_error(WAN_EALIGN, "ctx not 16-byte aligned");
-  if (ctx_lens && !aligned16(ctx_lens)) return set_error(WAN_EALIGN, "ctx_lens not 16-byte aligned");
-  const int gmax = d.F > d.H ? (d.F > d.W ? d.F : d.W) : (d.H > d.W ? d.H : d.W);
-  if (rope_max_pos < gmax) return set_error(WAN_EINVAL, "rope table has %d rows, grid needs %d", rope_max_pos, gmax);
-  const WsLayout lay = layout_of(dims, B);
-  if (ws_bytes < lay.total) return set_error(WAN_EINVAL, "workspace %zu bytes < %zu needed", ws_bytes, lay.total);
-
-  char *ws = static_cast<char *>(workspace);
-  void *act = ws + lay.off[WAN_WS_ACT];
-  char *qkv = ws + lay.off[WAN_WS_QKV];
-  void *o = ws + lay.off[WAN_WS_O];
-  void *qc = ws + lay.off[WAN_WS_QC];
-  char *kvc = ws + lay.off[WAN_WS_KVC];
-  void *oc = ws + lay.off[WAN_WS_OC];
-  void *hbuf = ws + lay.off[WAN_WS_H];
-  float *mod = reinterpret_cast<float *>(ws + lay.off[WAN_WS_MOD]);
-  const int BL = B * L;
-
-  // m = modulation + e0  (shift, scale, gate, shift2, scale2, gate2)
-  const ModSrc ms{d.e0_per_token != 0, e0, mod, w->modulation, L, D};
-  if (!ms.ptok && (rc = WAN_PROF(WAN_K_MISC, s, launch_mod_combine(w->modulation, e0, mod, B, D, s)))) return rc;
-  if (is_fp8(dt)) return block_forward_fp8(d, B, x, ctx, ctx_lens, w, rope, ws, lay, ms, s);
-
-  // ---- self-attention branch: x += m2 * Wo . Attn(RoPE(RMSNorm(q,k)), v)
-  // bf16 tensor-core path: the QKV GEMM epilogue accumulates each row's sum of
-  // squares of q and k, writes gamma * RoPE(y); the attention applies q's RMS
-  // factor in its logit scale and a row pass applies k's. Otherwise: plain
-  // GEMM, then an RMSNorm + RoPE pass over q and k.
-  float *stats = reinterpret_cast<float *>(ws + lay.off[WAN_WS_STATS]);
-  GemmArgs gqkv = {};
-  gqkv.M = BL; gqkv.N = 3 * D; gqkv.K = D; gqkv.A = act; gqkv.lda = D;
-  gqkv.Bseg[0] = w->wq; gqkv.Bseg[1] = w->wk; gqkv.Bseg[2] = w->wv;
-  gqkv.bias[0] = w->bq; gqkv.bias[1] = w->bk; gqkv.bias[2] = w->bv;
-  gqkv.segN = D; gqkv.nseg = 3; gqkv.C = qkv; gqkv.ldc = 3 * D;
-  gqkv.epi = EPI_QKNORM;
-  gqkv.gamma[0] = w->gq; gqkv.gamma[1] = w->gk; gqkv.gamma[2] = nullptr;
-  const int parts = D >= 256 ? D / 256 : 1;          // partial sums per row (one per 256-column tile)
-  const int sstride = 4 * parts;                      // q | k | cross q | cross k partials of a row
-  gqkv.ss = stats; gqkv.ss_stride = sstride; gqkv.ss_col[0] = 0; gqkv.ss_col[1] = 1; gqkv.ss_col[2] = -1;
-  gqkv.rope = rope; gqkv.rope_mask = 3; gqkv.F = d.F; gqkv.H = d.H; gqkv.W = d.W; gqkv.head_dim = hd;
-  AttnArgs aself = {};
-  aself.B = B; aself.heads = d.heads; aself.Lq = L; aself.Lk = L; aself.d = hd;
-  aself.q = qkv; aself.ldq = 3 * D; aself.k = qkv + D * es; aself.ldk = 3 * D; aself.v = qkv + 2 * D * es; aself.ldv = 3 * D;
-  aself.o = o; aself.ldo = D; aself.k_lens = nullptr; aself.scale = 1.0f / sqrtf((float)hd);
-  const bool fused = dt == WAN_BF16;
-  if (fused && !(gemm_tc_supported(gqkv) && attention_tc_supported(aself)))
-    return set_error(WAN_EUNSUPPORTED, "bf16 block: the QKV GEMM or the self-attention is outside the "
-                                       "tensor-core kernels' rules (dim %% 256 == 0, head_dim 128)");
-
-  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, ln_of(ms, 0, 1), nullptr, nullptr, d.eps, s)))) return rc;
-  if (fused) {
-    if ((rc = run_gemm(gqkv, dt, s))) return rc;
-    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_scale_rows(qkv + D * es, BL, 3 * D, D, stats + parts, sstride, parts, d.eps, s)))) return rc;
-    aself.q_ss = stats; aself.q_ss_stride = sstride; aself.q_ss_parts = parts; aself.q_ss_n = (float)D; aself.q_ss_eps = d.eps;
-  } else {
-    gqkv.epi = EPI_STORE;
-    if ((rc = run_gemm(gqkv, dt, s))) return rc;
-    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qkv, dt, BL, 3 * D, D, hd, w->gq, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s)))) return rc;
-    if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qkv + D * es, dt, BL, 3 * D, D, hd, w->gk, d.eps, rope, rope_max_pos, d.F, d.H, d.W, s)))) return rc;
-  }
-  if ((rc = run_attention(aself, dt, s, WAN_K_ATTN_SELF))) return rc;
-  {
-    GemmArgs g = {};
-    g.M = BL; g.N = D; g.K = D; g.A = o; g.lda = D;
-    g.Bseg[0] = w->wo; g.bias[0] = w->bo; g.segN = D; g.nseg = 1;
-    g.epi = EPI_RESID; g.X = x; g.ldx = D;
-    gate_of(ms, g, 2);
-    if ((rc = run_gemm(g, dt, s))) return rc;
-  }
-
-  // ---- cross-attention branch (ungated): x += Wco . Attn(q(norm3 x), k(ctx), v(ctx))
-  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, LnMod{}, w->g3, w->b3, d.eps, s)))) return rc;
-  {
-    GemmArgs g = {};
-    g.M = BL; g.N = D; g.K = D; g.A = act; g.lda = D;
-    g.Bseg[0] = w->cwq; g.bias[0] = w->cbq; g.segN = D; g.nseg = 1;
-    g.C = qc; g.ldc = D;
-    g.epi = fused ? EPI_QKNORM : EPI_STORE;
-    g.gamma[0] = w->cgq; g.ss = stats; g.ss_stride = sstride; g.ss_col[0] = 2; g.ss_col[1] = g.ss_col[2] = -1;
-    if ((rc = run_gemm(g, dt, s))) return rc;
-  }
-  if (!fused && (rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(qc, dt, BL, D, D, hd, w->cgq, d.eps, nullptr, 0, 1, 1, 1, s)))) return rc;
-  if (T > 0) {
-    GemmArgs g = {};
-    g.M = B * T; g.N = 2 * D; g.K = D; g.A = ctx; g.lda = D;
-    g.Bseg[0] = w->cwk; g.Bseg[1] = w->cwv; g.bias[0] = w->cbk; g.bias[1] = w->cbv;
-    g.segN = D; g.nseg = 2; g.C = kvc; g.ldc = 2 * D;
-    g.epi = fused ? EPI_QKNORM : EPI_STORE;
-    g.gamma[0] = w->cgk; g.gamma[1] = nullptr; g.ss = stats; g.ss_stride = sstride;
-    g.ss_col[0] = 3; g.ss_col[1] = -1; g.ss_col[2] = -1;
-    if ((rc = run_gemm(g, dt, s))) return rc;
-    if (fused) {
-      if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_scale_rows(kvc, B * T, 2 * D, D, stats + 3 * parts, sstride, parts, d.eps, s)))) return rc;
-    } else if ((rc = WAN_PROF(WAN_K_QKNORM_ROPE, s, launch_rmsnorm_rope(kvc, dt, B * T, 2 * D, D, hd, w->cgk, d.eps, nullptr, 0, 1, 1, 1, s)))) {
-      return rc;
-    }
-  }
-  {
-    AttnArgs a = {};
-    a.B = B; a.heads = d.heads; a.Lq = L; a.Lk = T; a.d = hd;
-    a.q = qc; a.ldq = D; a.k = kvc; a.ldk = 2 * D; a.v = kvc + D * es; a.ldv = 2 * D;
-    a.o = oc; a.ldo = D; a.k_lens = ctx_lens; a.scale = 1.0f / sqrtf((float)hd);
-    if (fused) {
-      a.q_ss = stats + 2 * parts; a.q_ss_stride = sstride; a.q_ss_parts = parts;
-      a.q_ss_n = (float)D; a.q_ss_eps = d.eps;
-    }
-    if ((rc = run_attention(a, dt, s, WAN_K_ATTN_CROSS))) return rc;
-  }
-  {
-    GemmArgs g = {};
-    g.M = BL; g.N = D; g.K = D; g.A = oc; g.lda = D;
-    g.Bseg[0] = w->cwo; g.bias[0] = w->cbo; g.segN = D; g.nseg = 1;
-    g.epi = EPI_RESID; g.X = x; g.ldx = D; g.gate = nullptr; g.rows_per_gate = L;
-    if ((rc = run_gemm(g, dt, s))) return rc;
-  }
-
-  // ---- FFN branch: x += m5 * W2 . gelu_tanh(W1 . (LN(x)(1 + m4) + m3))
-  if ((rc = WAN_PROF(WAN_K_LAYERNORM, s, launch_layernorm_mod(x, act, dt, BL, D, ln_of(ms, 3, 4), nullptr, nullptr, d.eps, s)))) return rc;
-  {
-    GemmArgs g = {};
-    g.M = BL; g.N = Fh; g.K = D; g.A = act; g.lda = D;
-    g.Bseg[0] = w->w1; g.bias[0] = w->b1; g.segN = Fh; g.nseg = 1;
-    g.epi = EPI_GELU; g.C = hbuf; g.ldc = Fh;
-    if ((rc = run_gemm(g, dt, s))) return rc;
-  }
-  {
-    GemmArgs g = {};
-    g.M = BL; g.N = D; g.K = Fh; g.A = hbuf; g.lda = Fh;
-    g.Bseg[0] = w->w2; g.bias[0] = w->b2; g.segN = D; g.nseg = 1;
-    g.epi = EPI_RESID; g.X = x; g.ldx = D;
-    gate_of(ms, g, 5);
-    if ((rc = run_gemm(g, dt, s))) return rc;
-  }
-  return WAN_OK;
+  return WAN_PROF(WAN_K_MISC, s, launch_permute_chunks(src, dst, ndim, dims, perm, chunk_bytes, s));
 }
 
 int wan_quantize_fp8(const void *src, int src_dtype, int rows, int cols, int per_row, uint8_t *q,

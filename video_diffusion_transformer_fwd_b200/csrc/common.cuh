@@ -107,7 +107,8 @@ enum Epilogue { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_QKNORM = 3, EPI_
 //              ss_col[s] >= 0, the sum of y^2 over each 256-column tile t of the
 //              segment is written to ss[m * ss_stride + ss_col[s] * (segN / 256) + t]
 //              (the consumer adds the segN / 256 partials of a row),
-//              and C = gamma[s] * y, rotated by the 3D RoPE of token m % L when
+//              and C = gamma[s] * y, rotated by the 3D RoPE of token
+//              tok0 + m % rows_per_seq when
 //              bit s of rope_mask is set; otherwise C = y. The row's RMS factor
 //              is applied later (attention logit scale for q, a row pass for k).
 struct GemmArgs {
@@ -125,6 +126,9 @@ struct GemmArgs {
   const float *b_scale[3];  // one device float per weight segment
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
   const float *rope; int rope_mask; int F, H, W; int head_dim;
+  // rows of A per sequence (0: F*H*W) and the grid index of a sequence's
+  // first row: row m is token tok0 + m % rows_per_seq of the (F, H, W) grid
+  int rows_per_seq, tok0;
 };
 
 int gemm_simt(const GemmArgs &g, int dtype, cudaStream_t s);
@@ -187,10 +191,11 @@ int launch_quant_rows(const void *src, int dtype, size_t ld, int rows, int cols,
                       cudaStream_t s);
 int launch_quant_tensor(const void *src, int dtype, size_t n, uint8_t *q, float *scale, cudaStream_t s);
 // In place on rows of a strided matrix: v = RMSNorm_D(v) * gain, then the 3D
-// RoPE of token (r % L) when rope != NULL.
+// RoPE of token tok0 + r % rows_per_seq of the (F, H, W) grid when rope != NULL
+// (rows_per_seq 0: F*H*W).
 int launch_rmsnorm_rope(void *p, int dtype, int rows, int ld, int D, int head_dim,
                         const float *gain, float eps, const float *rope, int rope_max_pos,
-                        int F, int H, int W, cudaStream_t s);
+                        int F, int H, int W, cudaStream_t s, int rows_per_seq = 0, int tok0 = 0);
 // In place 3D RoPE only (no norm), rows of a [rows, heads*d] strided matrix.
 int launch_rope_only(void *p, int dtype, int rows, int ld, int D, int head_dim,
                      const float *rope, int rope_max_pos, int F, int H, int W, cudaStream_t s);
@@ -199,6 +204,10 @@ int launch_rope_only(void *p, int dtype, int rows, int ld, int D, int head_dim,
 int launch_scale_rows(void *p, int rows, int ld, int D, const float *ss, int ss_stride, int parts,
                       float eps, cudaStream_t s);
 int launch_rope_table(int head_dim, int max_pos, double theta, float *table, cudaStream_t s);
+// dst = src with its chunk axes permuted: src is [dims[0]] ... [dims[nd-1]]
+// chunks of chunk_bytes, dst axis k runs over src axis perm[k].
+int launch_permute_chunks(const void *src, void *dst, int nd, const int *dims, const int *perm,
+                          size_t chunk_bytes, cudaStream_t s);
 int launch_euler_cfg(float *x, const void *vc, const void *vu, int vdt, size_t n, float scale,
                      float dt, cudaStream_t s);
 

@@ -404,7 +404,7 @@ template <typename T, bool NORM, bool ROPE>
 __global__ void __launch_bounds__(LN_THREADS)
 rmsnorm_rope_kernel(T *__restrict__ p, int ld, int D, int head_dim,
                     const float *__restrict__ gain, float eps, const float *__restrict__ rope,
-                    int L, int H, int W) {
+                    int L, int H, int W, int tok0) {
   __shared__ float red[32];
   const int row = blockIdx.x;
   T *pr = p + (size_t)row * ld;
@@ -423,7 +423,7 @@ rmsnorm_rope_kernel(T *__restrict__ p, int ld, int D, int head_dim,
   if (NORM) r = 1.0f / sqrtf(block_sum(ss, red) / (float)D + eps);
   int tpos = 0, hpos = 0, wpos = 0, half = head_dim >> 1, c3 = half / 3, pt = half - 2 * c3;
   if (ROPE) {
-    const int tok = row % L;
+    const int tok = tok0 + row % L;
     tpos = tok / (H * W);
     hpos = (tok / W) % H;
     wpos = tok % W;
@@ -451,26 +451,27 @@ rmsnorm_rope_kernel(T *__restrict__ p, int ld, int D, int head_dim,
 
 template <bool NORM, bool ROPE>
 static int launch_rr(void *p, int dtype, int rows, int ld, int D, int head_dim, const float *gain,
-                     float eps, const float *rope, int L, int H, int W, cudaStream_t s) {
+                     float eps, const float *rope, int L, int H, int W, int tok0, cudaStream_t s) {
   if (dtype == WAN_BF16)
     rmsnorm_rope_kernel<__nv_bfloat16, NORM, ROPE><<<rows, LN_THREADS, 0, s>>>(
-        (__nv_bfloat16 *)p, ld, D, head_dim, gain, eps, rope, L, H, W);
+        (__nv_bfloat16 *)p, ld, D, head_dim, gain, eps, rope, L, H, W, tok0);
   else
     rmsnorm_rope_kernel<float, NORM, ROPE><<<rows, LN_THREADS, 0, s>>>(
-        (float *)p, ld, D, head_dim, gain, eps, rope, L, H, W);
+        (float *)p, ld, D, head_dim, gain, eps, rope, L, H, W, tok0);
   WAN_CHECK_LAUNCH("rmsnorm_rope");
   return WAN_OK;
 }
 
 int launch_rmsnorm_rope(void *p, int dtype, int rows, int ld, int D, int head_dim,
                         const float *gain, float eps, const float *rope, int rope_max_pos,
-                        int F, int H, int W, cudaStream_t s) {
+                        int F, int H, int W, cudaStream_t s, int rows_per_seq, int tok0) {
   (void)rope_max_pos;
   if (D % 4 || D > 4 * LN_MAXV * LN_THREADS || head_dim % 4)
     return set_error(WAN_EUNSUPPORTED, "rmsnorm_rope: D=%d head_dim=%d", D, head_dim);
   if (rows == 0) return WAN_OK;
-  if (rope) return launch_rr<true, true>(p, dtype, rows, ld, D, head_dim, gain, eps, rope, F * H * W, H, W, s);
-  return launch_rr<true, false>(p, dtype, rows, ld, D, head_dim, gain, eps, nullptr, 1, 1, 1, s);
+  const int L = rows_per_seq > 0 ? rows_per_seq : F * H * W;
+  if (rope) return launch_rr<true, true>(p, dtype, rows, ld, D, head_dim, gain, eps, rope, L, H, W, tok0, s);
+  return launch_rr<true, false>(p, dtype, rows, ld, D, head_dim, gain, eps, nullptr, 1, 1, 1, 0, s);
 }
 
 int launch_rope_only(void *p, int dtype, int rows, int ld, int D, int head_dim,
@@ -479,7 +480,57 @@ int launch_rope_only(void *p, int dtype, int rows, int ld, int D, int head_dim,
   if (D % 4 || D > 4 * LN_MAXV * LN_THREADS || head_dim % 4)
     return set_error(WAN_EUNSUPPORTED, "rope: D=%d head_dim=%d", D, head_dim);
   if (rows == 0) return WAN_OK;
-  return launch_rr<false, true>(p, dtype, rows, ld, D, head_dim, nullptr, 0.f, rope, F * H * W, H, W, s);
+  return launch_rr<false, true>(p, dtype, rows, ld, D, head_dim, nullptr, 0.f, rope, F * H * W, H, W, 0, s);
+}
+
+// ----------------------------------------------------------------------------
+// Chunk permutation around the all-to-all of the head-parallel attention:
+// src holds prod(dims) chunks of chunk_bytes in row-major order of `dims`;
+// dst chunk (j_0, ..., j_{nd-1}) (row-major over dims[perm[k]]) is src chunk
+// i with i[perm[k]] = j_k. One 16-byte vector per thread, grid-stride.
+// ----------------------------------------------------------------------------
+struct PermuteArgs {
+  int nd;
+  long long dst_ext[5];       // extent of dst axis k (= dims[perm[k]])
+  long long src_stride[5];    // src chunk stride of the src axis that dst axis k runs over
+};
+
+__global__ void permute_chunks_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, PermuteArgs a,
+                                      long long vpc, long long total) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long chunk = i / vpc, v = i - chunk * vpc;
+    long long rem = chunk, off = 0;
+    for (int k = a.nd - 1; k >= 0; --k) {
+      const long long j = rem % a.dst_ext[k];
+      rem /= a.dst_ext[k];
+      off += j * a.src_stride[k];
+    }
+    dst[i] = src[off * vpc + v];
+  }
+}
+
+int launch_permute_chunks(const void *src, void *dst, int nd, const int *dims, const int *perm,
+                          size_t chunk_bytes, cudaStream_t s) {
+  PermuteArgs a = {};
+  a.nd = nd;
+  long long stride[5], nchunks = 1;
+  for (int k = nd - 1; k >= 0; --k) {
+    stride[k] = nchunks;
+    nchunks *= dims[k];
+  }
+  for (int k = 0; k < nd; ++k) {
+    a.dst_ext[k] = dims[perm[k]];
+    a.src_stride[k] = stride[perm[k]];
+  }
+  const long long vpc = (long long)(chunk_bytes / 16), total = nchunks * vpc;
+  if (total == 0) return WAN_OK;
+  const long long want = (total + 255) / 256;
+  const int blocks = (int)(want < 148LL * 16 ? want : 148LL * 16);
+  permute_chunks_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(src), static_cast<uint4 *>(dst), a,
+                                               vpc, total);
+  WAN_CHECK_LAUNCH("permute_chunks");
+  return WAN_OK;
 }
 
 // ----------------------------------------------------------------------------

@@ -62,7 +62,7 @@ struct TcParams {
   const float *a_scale; const float *b_scale[3];      // FP8: per row of A, per weight segment
   // q/k RMSNorm + RoPE epilogue (EPI_QKNORM)
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
-  const float *rope; int rope_mask; int L, H, W; int head_dim;
+  const float *rope; int rope_mask; int L, H, W; int head_dim; int tok0;   // L: rows per sequence
   int *watchdog;
 };
 
@@ -245,7 +245,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         ss_col = p.ss_col[seg];
         gam = p.gamma[seg];
         do_rope = (p.rope_mask >> seg) & 1;
-        const int tok = (m < p.M ? m : 0) % p.L;
+        const int tok = p.tok0 + (m < p.M ? m : 0) % p.L;
         tpos = tok / (p.H * p.W);
         hpos = (tok / p.W) % p.H;
         wpos = tok % p.W;
@@ -475,7 +475,9 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   }
   p.ss = g.ss; p.ss_stride = g.ss_stride;
   p.rope = g.rope; p.rope_mask = g.rope ? g.rope_mask : 0;
-  p.L = g.F * g.H * g.W > 0 ? g.F * g.H * g.W : 1; p.H = g.H > 0 ? g.H : 1; p.W = g.W > 0 ? g.W : 1;
+  p.L = g.rows_per_seq > 0 ? g.rows_per_seq : (g.F * g.H * g.W > 0 ? g.F * g.H * g.W : 1);
+  p.H = g.H > 0 ? g.H : 1; p.W = g.W > 0 ? g.W : 1;
+  p.tok0 = g.tok0;
   p.head_dim = g.head_dim > 0 ? g.head_dim : 128;
   p.watchdog = watchdog_ptr();
   CUtensorMap tx = ta;

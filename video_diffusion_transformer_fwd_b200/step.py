@@ -140,6 +140,174 @@ class CFGParallelStep:
                                              c.sigma_next, wan._stream(stream)))
         return self.x
 
+def permute_chunks_device(src, dst, dims, perm, chunk_bytes, stream=None):
+    """dst = src with its chunk axes permuted, by wan_permute_chunks."""
+    wan.check(wan.wan_permute_chunks(src.data_ptr(), dst.data_ptr(), len(dims), dims, perm, chunk_bytes,
+                                     wan._stream(stream)))
+
+
+def seq_head_exchange(send, recv, group):
+    """The all-to-all of the head-parallel attention: ``send`` and ``recv``
+    are [N, ...] with block j of ``send`` going to rank j of ``group`` and
+    block i of ``recv`` coming from rank i. NCCL moves device buffers
+    directly (over NVLink between GPUs of one node); other backends stage
+    through host memory."""
+    import torch.distributed as dist
+    if dist.get_backend(group) == "nccl":
+        dist.all_to_all_single(recv, send, group=group)
+    else:
+        r = torch.empty(recv.shape, dtype=recv.dtype)
+        dist.all_to_all_single(r, send.cpu(), group=group)
+        recv.copy_(r)
+
+
+class UlyssesExchange:
+    """Buffers and layout changes of the head-parallel (Ulysses) attention
+    for one of N ranks ("Wan paper deep dive" (charles2530.github.io),
+    training/inference-system section: Ulysses inside Ring). Rank r holds
+    tokens [r rows, (r + 1) rows) of each of B sequences and, between the
+    two all-to-alls, heads [r hl, (r + 1) hl) of all L = N rows tokens
+    (hl = heads / N). Layouts (chunks of hl * d elements):
+
+      q|k|v rows  [B][rows][3][N][hl d]    (wan_block_sp_qkv output)
+      send_qkv    [N][B][rows][3][hl d]    block j -> rank j
+      recv_qkv    [N][B][rows][3][hl d]    block i <- rank i (tokens of shard i)
+      qkv_heads   [3][B][N rows][hl d]     dense q, k, v of this rank's heads
+      o_heads     [B][N rows][hl d]        attention output, this rank's heads
+      send_o      [N][B][rows][hl d]       tokens of shard j -> rank j
+      recv_o      [N][B][rows][hl d]       heads of rank i
+      o_rows      [B][rows][N][hl d]       all heads of this rank's rows
+
+    ``permute`` and ``exchange`` default to wan_permute_chunks and
+    seq_head_exchange; tests pass host versions."""
+
+    def __init__(self, B, L, N, heads, head_dim, dtype, group=None, device="cuda", permute=None,
+                 exchange=None):
+        if N < 1 or L % N or heads % N:
+            raise ValueError(f"{N} ranks must divide the {L} tokens and the {heads} heads")
+        self.B, self.L, self.N, self.rows, self.hl, self.d = B, L, N, L // N, heads // N, head_dim
+        self.group = group
+        self.permute = permute or permute_chunks_device
+        self.exchange = exchange or seq_head_exchange
+        c = self.hl * head_dim
+        self.chunk_elems = c
+        self.chunk_bytes = c * torch.empty((), dtype=dtype).element_size()
+        B, rows = self.B, self.rows
+        mk = lambda *shape: torch.empty(shape, dtype=dtype, device=device)
+        self.qkv_rows = mk(B, rows, 3 * N * c)
+        self.send_qkv = mk(N, B, rows, 3, c)
+        self.recv_qkv = mk(N, B, rows, 3, c)
+        self.qkv_heads = mk(3, B, N * rows, c)
+        self.o_heads = mk(B, N * rows, c)
+        self.send_o = mk(N, B, rows, c)
+        self.recv_o = mk(N, B, rows, c)
+        self.o_rows = mk(B, rows, N * c)
+
+    def pack_qkv(self, stream=None):
+        self.permute(self.qkv_rows, self.send_qkv, (self.B, self.rows, 3, self.N), (3, 0, 1, 2),
+                     self.chunk_bytes, stream)
+
+    def unpack_qkv(self, stream=None):
+        self.permute(self.recv_qkv, self.qkv_heads, (self.N, self.B, self.rows, 3), (3, 1, 0, 2),
+                     self.chunk_bytes, stream)
+
+    def pack_o(self, stream=None):
+        self.permute(self.o_heads, self.send_o, (self.B, self.N, self.rows), (1, 0, 2), self.chunk_bytes, stream)
+
+    def unpack_o(self, stream=None):
+        self.permute(self.recv_o, self.o_rows, (self.N, self.B, self.rows), (1, 2, 0), self.chunk_bytes, stream)
+
+    def to_heads(self, stream=None):
+        """qkv_rows (this rank's tokens, all heads) -> qkv_heads (all tokens,
+        this rank's heads)."""
+        self.pack_qkv(stream)
+        self.exchange(self.send_qkv, self.recv_qkv, self.group)
+        self.unpack_qkv(stream)
+
+    def to_rows(self, stream=None):
+        """o_heads (all tokens, this rank's heads) -> o_rows (this rank's
+        tokens, all heads)."""
+        self.pack_o(stream)
+        self.exchange(self.send_o, self.recv_o, self.group)
+        self.unpack_o(stream)
+
+
+class UlyssesStep:
+    """The denoising step of DenoiseStep with every block's self-attention
+    head-parallel over the N ranks of ``group``: rank r keeps tokens
+    [r L/N, (r + 1) L/N) of x (and of the CFG pair's block inputs), runs
+    wan_block_sp_qkv on them, exchanges q, k, v so that it holds all tokens
+    of heads [r n/N, (r + 1) n/N), runs wan_attention on those, exchanges the
+    outputs back and runs wan_block_sp_finish on its tokens. The CFG-Euler
+    update is elementwise, so each rank moves its own tokens. With the same
+    seed the inputs and weights are those of DenoiseStep; no kernel mixes
+    tokens of different shards except the attention, which sees whole
+    sequences, so the union of the ranks' x equals the single-rank phase
+    path (N = 1) bit for bit."""
+
+    def __init__(self, cfg: BlockConfig, rank: int, N: int, group=None, seed: int = 0, device: str = "cuda",
+                 weights=None, exchange=None):
+        if cfg.L % N or cfg.heads % N:
+            raise ValueError(f"{N} ranks must divide L = {cfg.L} and heads = {cfg.heads}")
+        self.cfg, self.rank, self.N = cfg, rank, N
+        self.rows = cfg.L // N
+        self.tok0 = rank * self.rows
+        self.dims = wan.dims_of(cfg)
+        self.weights = weights if weights is not None else synth.step_weights(cfg, device, seed)
+        self.cweights = [wan.make_weights(w) for w in self.weights]
+        acts = synth.block_activations(2, cfg.L, cfg.dim, cfg.text_len, cfg.dtype, device, seed + 100,
+                                       same_e0=True)
+        self.x = acts["x"][0, self.tok0:self.tok0 + self.rows].contiguous()   # [rows, D], this shard
+        self.ctx = acts["ctx"]
+        self.e0 = acts["e0"]
+        del acts
+        self.xb = torch.empty((2, self.rows, cfg.dim), dtype=torch.float32, device=device)
+        self.rope = wan.rope_freqs(cfg.head_dim, 1024, cfg.theta, device=device)
+        n = wan.wan_block_sp_workspace_bytes(self.dims, 2, self.rows)
+        if n == 0:
+            raise wan.WanError(wan.WAN_EINVAL, wan.last_error())
+        self.ws = torch.empty(n, dtype=torch.uint8, device=device)
+        self.ex = UlyssesExchange(2, cfg.L, N, cfg.heads, cfg.head_dim, synth.TORCH_DTYPES[cfg.dtype], group,
+                                  device, exchange=exchange)
+        self.hl = cfg.heads // N
+
+    def block_qkv(self, i, stream=None):
+        wan.check(wan.wan_block_sp_qkv(self.dims, 2, self.rows, self.tok0, self.xb.data_ptr(), self.e0.data_ptr(),
+                                       self.cweights[i], self.rope.data_ptr(), self.rope.shape[0],
+                                       self.ex.qkv_rows.data_ptr(), self.ws.data_ptr(), self.ws.numel(),
+                                       wan._stream(stream)))
+
+    def block_attention(self, stream=None):
+        q, k, v = self.ex.qkv_heads[0], self.ex.qkv_heads[1], self.ex.qkv_heads[2]
+        c = self.cfg
+        wan.check(wan.wan_attention(2, self.hl, c.L, c.L, c.head_dim, self.dims.dtype, q.data_ptr(), k.data_ptr(),
+                                    v.data_ptr(), self.ex.o_heads.data_ptr(), None, 0.0, None, None, 0,
+                                    wan._stream(stream)))
+
+    def block_finish(self, i, stream=None):
+        wan.check(wan.wan_block_sp_finish(self.dims, 2, self.rows, self.xb.data_ptr(), self.ctx.data_ptr(), None,
+                                          self.e0.data_ptr(), self.cweights[i], self.ex.o_rows.data_ptr(),
+                                          self.ws.data_ptr(), self.ws.numel(), wan._stream(stream)))
+
+    def euler(self, stream=None):
+        c = self.cfg
+        wan.check(wan.wan_euler_cfg_step(self.x.data_ptr(), self.xb[0].data_ptr(), self.xb[1].data_ptr(),
+                                         wan.WAN_F32, self.x.numel(), c.guide_scale, c.sigma, c.sigma_next,
+                                         wan._stream(stream)))
+
+    def step(self, stream=None):
+        self.xb[0].copy_(self.x)
+        self.xb[1].copy_(self.x)
+        for i in range(len(self.cweights)):
+            self.block_qkv(i, stream)
+            self.ex.to_heads(stream)
+            self.block_attention(stream)
+            self.ex.to_rows(stream)
+            self.block_finish(i, stream)
+        self.euler(stream)
+        return self.x
+
+
 class ModelDenoiseStep:
     """One CFG flow-matching Euler step on the latent through the whole model
     (wan_model_forward on the CFG pair at t = 1000 sigma, then

@@ -80,6 +80,13 @@ _SIGS = {
                                    ctypes.POINTER(wan_block_weights), _vp, _c_int, _vp, _sz, _vp]),
     "wan_block_forward_noalloc": (_c_int, [ctypes.POINTER(wan_dims), _c_int, _vp, _vp, _vp, _vp,
                                            ctypes.POINTER(wan_block_weights), _vp, _c_int, _vp]),
+    "wan_block_sp_workspace_bytes": (_sz, [ctypes.POINTER(wan_dims), _c_int, _c_int]),
+    "wan_block_sp_qkv": (_c_int, [ctypes.POINTER(wan_dims), _c_int, _c_int, _c_int, _vp, _vp,
+                                  ctypes.POINTER(wan_block_weights), _vp, _c_int, _vp, _vp, _sz, _vp]),
+    "wan_block_sp_finish": (_c_int, [ctypes.POINTER(wan_dims), _c_int, _c_int, _vp, _vp, _vp, _vp,
+                                     ctypes.POINTER(wan_block_weights), _vp, _vp, _sz, _vp]),
+    "wan_permute_chunks": (_c_int, [_vp, _vp, _c_int, ctypes.POINTER(ctypes.c_int),
+                                    ctypes.POINTER(ctypes.c_int), _sz, _vp]),
     "wan_attention": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _vp, _vp, _vp, _vp,
                                _vp, ctypes.c_float, ctypes.POINTER(ctypes.c_int), _vp, _c_int, _vp]),
     "wan_euler_cfg_step": (_c_int, [_vp, _vp, _vp, _c_int, _sz, ctypes.c_float, ctypes.c_float,
@@ -160,6 +167,27 @@ def wan_block_forward(dims, B, x, ctx, ctx_lens, e0, weights, rope, rope_max_pos
 def wan_block_forward_noalloc(dims, B, x, ctx, ctx_lens, e0, weights, rope, rope_max_pos, stream):
     return load().wan_block_forward_noalloc(ctypes.byref(dims), B, x, ctx, ctx_lens, e0,
                                             ctypes.byref(weights), rope, rope_max_pos, stream)
+
+
+def wan_block_sp_workspace_bytes(dims, B, rows):
+    return load().wan_block_sp_workspace_bytes(ctypes.byref(dims), B, rows)
+
+
+def wan_block_sp_qkv(dims, B, rows, tok0, x, e0, weights, rope, rope_max_pos, qkv, workspace, ws_bytes,
+                     stream):
+    return load().wan_block_sp_qkv(ctypes.byref(dims), B, rows, tok0, x, e0, ctypes.byref(weights), rope,
+                                   rope_max_pos, qkv, workspace, ws_bytes, stream)
+
+
+def wan_block_sp_finish(dims, B, rows, x, ctx, ctx_lens, e0, weights, o, workspace, ws_bytes, stream):
+    return load().wan_block_sp_finish(ctypes.byref(dims), B, rows, x, ctx, ctx_lens, e0, ctypes.byref(weights),
+                                      o, workspace, ws_bytes, stream)
+
+
+def wan_permute_chunks(src, dst, ndim, dims, perm, chunk_bytes, stream):
+    d = (ctypes.c_int * max(ndim, 1))(*dims)
+    p = (ctypes.c_int * max(ndim, 1))(*perm)
+    return load().wan_permute_chunks(src, dst, ndim, d, p, chunk_bytes, stream)
 
 
 def wan_attention(B, heads, Lq, Lk, head_dim, dtype, q, k, v, o, k_lens, scale, grid, rope,
