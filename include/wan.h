@@ -47,6 +47,7 @@ typedef struct CUstream_st *wan_stream_t;
 #define WAN_EUNSUPPORTED -3   /* dtype / head_dim combination not implemented           */
 #define WAN_ECUDA        -4   /* a CUDA runtime or driver call failed                   */
 #define WAN_ETIMEOUT     -5   /* a kernel's bounded wait gave up (see wan_device_status) */
+#define WAN_EBOUNDS      -6   /* debug builds: a kernel's store fell outside its buffer */
 
 /* element types */
 #define WAN_F32  0
@@ -454,8 +455,17 @@ int wan_euler_cfg_step(float *x, const void *v_cond, const void *v_uncond,
 /* wan_device_status -- synchronise `stream`, then report and clear the
  * library's device-side watchdog word for the current device: WAN_OK, or
  * WAN_ETIMEOUT if a kernel gave up a bounded wait since the last call (its
- * outputs are then invalid), or WAN_ECUDA if the stream holds a CUDA error. */
+ * outputs are then invalid), WAN_EBOUNDS if a debug build's bounds check
+ * caught a store outside its buffer (the store was skipped), or WAN_ECUDA if
+ * the stream holds a CUDA error. */
 int wan_device_status(wan_stream_t stream);
+
+/* wan_debug_bounds -- 1 in a debug build (compiled with WAN_DEBUG_BOUNDS:
+ * every plain global store of the block's kernels -- the GEMM and attention
+ * epilogues, LayerNorm, RMSNorm / RoPE, the k / q row scaling, the chunk
+ * permutation, CFG-Euler -- is checked against its buffer's extent before
+ * it is made), 0 otherwise. */
+int wan_debug_bounds(void);
 
 /* wan_selftest_watchdog -- enqueue a one-CTA kernel whose bounded wait on an
  * mbarrier can never complete, so the wait gives up after its limit (about

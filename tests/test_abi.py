@@ -147,3 +147,11 @@ def test_bf16_block_outside_tensor_core_rules_is_refused(lib, kw):
     assert rc == wan.WAN_EUNSUPPORTED
     assert "256" in wan.last_error()
     assert wan.wan_block_workspace_bytes(d, 1) == 0
+
+
+def test_release_build_has_no_debug_checks(lib):
+    """The product library is the release build; the bounds-checking one is
+    libwan_debug.so, loaded only through WAN_LIBRARY."""
+    if os.environ.get("WAN_LIBRARY"):
+        pytest.skip("WAN_LIBRARY names another build")
+    assert wan.wan_debug_bounds() == 0

@@ -774,6 +774,8 @@ int wan_euler_cfg_step(float *x, const void *v_cond, const void *v_uncond, int v
                                                     sigma_next - sigma, s));
 }
 
+int wan_debug_bounds(void) { return kDebugBounds ? 1 : 0; }
+
 int wan_device_status(wan_stream_t stream) {
   g_msg[0] = 0;
   WAN_TRY_CUDA(cudaStreamSynchronize((cudaStream_t)stream), "stream synchronize");
@@ -784,6 +786,9 @@ int wan_device_status(wan_stream_t stream) {
   if (v != 0) {
     const int zero = 0;
     WAN_TRY_CUDA(cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice), "clear watchdog");
+    if (v >= WAN_DBG_CODE_BASE)
+      return set_error(WAN_EBOUNDS, "debug bounds check: a store fell outside its buffer (site %d)",
+                       v - WAN_DBG_CODE_BASE);
     return set_error(WAN_ETIMEOUT, "a kernel gave up a bounded wait (code %d)", v);
   }
   return WAN_OK;

@@ -109,8 +109,11 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(const AttnArgs a) {
   const float inv = (l > 0.f) ? 1.0f / l : 0.f;
   T *orow = static_cast<T *>(a.o) + (size_t)(b * a.Lq + r) * a.ldo + h * D;
 #pragma unroll
+  const T *o_hi = static_cast<const T *>(a.o) + (size_t)(a.B * a.Lq - 1) * a.ldo + (size_t)a.heads * D;
+#pragma unroll
   for (int c = 0; c < NC; ++c)
-    store4(orow + 16 * c + 4 * part, make_float4(o[c].x * inv, o[c].y * inv, o[c].z * inv, o[c].w * inv));
+    if (WAN_DBG_OK(orow + 16 * c + 4 * part, 4 * sizeof(T), a.o, o_hi, a.dbg, WAN_DBG_CODE_BASE + 12))
+      store4(orow + 16 * c + 4 * part, make_float4(o[c].x * inv, o[c].y * inv, o[c].z * inv, o[c].w * inv));
 }
 
 template <typename T>
@@ -132,7 +135,9 @@ int attention_simt(const AttnArgs &a, int dtype, cudaStream_t s) {
     return set_error(WAN_EUNSUPPORTED, "attention_simt: head_dim %d", a.d);
   if (a.B == 0 || a.Lq == 0 || a.heads == 0) return WAN_OK;
   if (a.heads > 65535 || a.B > 65535) return set_error(WAN_EINVAL, "attention: grid too large");
-  return dtype == WAN_BF16 ? launch_t<__nv_bfloat16>(a, s) : launch_t<float>(a, s);
+  AttnArgs ad = a;
+  if (!ad.dbg) ad.dbg = dbg_word();
+  return dtype == WAN_BF16 ? launch_t<__nv_bfloat16>(ad, s) : launch_t<float>(ad, s);
 }
 
 }  // namespace wan

@@ -49,6 +49,7 @@ struct FaParams {
   __nv_bfloat16 *o; int ldo;
   const float *q_ss; int q_ss_stride; int q_ss_parts; float q_ss_inv_n; float q_ss_eps;   // optional per-row RMS factor of q
   int *watchdog;
+  const void *o_hi; int *dbg;           // debug bounds checks: end of o
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -374,7 +375,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           u.y = pack_bf16(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
           u.z = pack_bf16(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
           u.w = pack_bf16(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
-          dst[e] = u;
+          if (WAN_DBG_OK(dst + e, 16, p.o, p.o_hi, p.dbg, WAN_DBG_CODE_BASE + 3)) dst[e] = u;
         }
       }
     }
@@ -417,6 +418,8 @@ int attention_tc(const AttnArgs &a, cudaStream_t s) {
   p.q_ss_inv_n = a.q_ss_n > 0.f ? 1.0f / a.q_ss_n : 0.f; p.q_ss_eps = a.q_ss_eps;
   p.o = static_cast<__nv_bfloat16 *>(a.o); p.ldo = a.ldo;
   p.watchdog = watchdog_ptr();
+  p.dbg = a.dbg ? a.dbg : dbg_word();
+  p.o_hi = static_cast<const char *>(a.o) + ((size_t)(a.B * a.Lq - 1) * a.ldo + (size_t)a.heads * D) * 2;
   dim3 grid((a.Lq + 2 * TQ - 1) / (2 * TQ), a.heads, a.B);
   attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tq, tk, tv, p);
   WAN_CHECK_LAUNCH("attention_tc");

@@ -28,6 +28,32 @@ int *watchdog_ptr();
     if (e_ != cudaSuccess) return ::wan::cuda_error(e_, what);          \
   } while (0)
 
+// ---------------------------------------------------------------- debug bounds checks
+// In a build with -DWAN_DEBUG_BOUNDS (build_lib.build(debug=True)) a kernel
+// checks, before each plain global store, that the bytes it writes lie inside
+// the extent [lo, hi) that the call's sizes give the buffer; on a violation
+// it records `code` in the device status word (the first one is kept), skips
+// the store, and wan_device_status returns WAN_EBOUNDS. In other builds the
+// check is the constant true and dbg_word() is NULL. (TMA stores and
+// reductions are clipped by their tensor maps and are not checked.)
+#ifdef WAN_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+__device__ __forceinline__ bool dbg_in(const void *p, size_t n, const void *lo, const void *hi, int *word,
+                                       int code) {
+  const char *c = static_cast<const char *>(p);
+  if (c >= static_cast<const char *>(lo) && c + n <= static_cast<const char *>(hi)) return true;
+  if (word) atomicCAS(word, 0, code);
+  return false;
+}
+#define WAN_DBG_OK(p, n, lo, hi, word, code) ::wan::dbg_in((p), (n), (lo), (hi), (word), (code))
+#else
+constexpr bool kDebugBounds = false;
+#define WAN_DBG_OK(p, n, lo, hi, word, code) true
+#endif
+// Status word the debug checks record into (NULL in other builds).
+inline int *dbg_word() { return kDebugBounds ? watchdog_ptr() : nullptr; }
+constexpr int WAN_DBG_CODE_BASE = 0x40000000;   // codes >= this are bounds violations (wait codes are < 0x10000)
+
 // ---------------------------------------------------------------- element access
 template <typename T> struct ElemIO;
 template <> struct ElemIO<float> {
@@ -129,6 +155,7 @@ struct GemmArgs {
   // rows of A per sequence (0: F*H*W) and the grid index of a sequence's
   // first row: row m is token tok0 + m % rows_per_seq of the (F, H, W) grid
   int rows_per_seq, tok0;
+  int *dbg;               // debug bounds checks: status word (dbg_word())
 };
 
 int gemm_simt(const GemmArgs &g, int dtype, cudaStream_t s);
@@ -151,6 +178,7 @@ struct AttnArgs {
   // optional per-query-row RMS factor folded into the logit scale:
   // scale_row = scale / sqrt(sum_{t < q_ss_parts} q_ss[row * q_ss_stride + t] / q_ss_n + q_ss_eps)
   const float *q_ss; int q_ss_stride; int q_ss_parts; float q_ss_n; float q_ss_eps;
+  int *dbg;               // debug bounds checks: status word (dbg_word())
 };
 int attention_simt(const AttnArgs &a, int dtype, cudaStream_t s);
 // 8-bit attention (attn8.cu): bf16 q, k, v, o with head_dim 128; quantizes

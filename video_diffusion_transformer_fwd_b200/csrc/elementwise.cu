@@ -255,7 +255,8 @@ template <typename OutT, int VPT>
 __global__ void __launch_bounds__(LN_THREADS, LN_CTAS_PER_SM)
 layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int rows, int D, const LnMod md,
                      const float *__restrict__ g, const float *__restrict__ beta, float eps,
-                     float *__restrict__ row_scale) {
+                     float *__restrict__ row_scale, int *dbg) {
+  const OutT *out_hi = out + (size_t)rows * D;
   __shared__ float red[2][32];
   const int nv = D >> 2;
   int row = blockIdx.x;
@@ -324,7 +325,8 @@ layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int ro
           v[i] = u;
           amax = fmaxf(amax, absmax4(u));
         } else {
-          store4(orow + 4 * c, u);
+          if (WAN_DBG_OK(orow + 4 * c, 4 * sizeof(OutT), out, out_hi, dbg, WAN_DBG_CODE_BASE + 4))
+            store4(orow + 4 * c, u);
         }
       }
     }
@@ -335,7 +337,7 @@ layernorm_mod_kernel(const float *__restrict__ x, OutT *__restrict__ out, int ro
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
         const int c = threadIdx.x + i * LN_THREADS;
-        if (c < nv) qr[c] = quant4(v[i], inv);
+        if (c < nv && WAN_DBG_OK(qr + c, 4, out, out_hi, dbg, WAN_DBG_CODE_BASE + 5)) qr[c] = quant4(v[i], inv);
       }
       if (threadIdx.x == 0) row_scale[row] = __fdiv_rn(amax, E4M3_MAX);
     }
@@ -348,7 +350,8 @@ template <typename OutT, int VPT>
 static void ln_launch(const float *x, OutT *out, int rows, int D, const LnMod &m, const float *g,
                       const float *beta, float eps, float *row_scale, cudaStream_t s) {
   const int grid = rows < LN_CTAS_PER_SM * sm_count() ? rows : LN_CTAS_PER_SM * sm_count();
-  layernorm_mod_kernel<OutT, VPT><<<grid, LN_THREADS, 0, s>>>(x, out, rows, D, m, g, beta, eps, row_scale);
+  layernorm_mod_kernel<OutT, VPT><<<grid, LN_THREADS, 0, s>>>(x, out, rows, D, m, g, beta, eps, row_scale,
+                                                               dbg_word());
 }
 
 template <typename OutT>
@@ -404,10 +407,11 @@ template <typename T, bool NORM, bool ROPE>
 __global__ void __launch_bounds__(LN_THREADS)
 rmsnorm_rope_kernel(T *__restrict__ p, int ld, int D, int head_dim,
                     const float *__restrict__ gain, float eps, const float *__restrict__ rope,
-                    int L, int H, int W, int tok0) {
+                    int L, int H, int W, int tok0, int rows, int *dbg) {
   __shared__ float red[32];
   const int row = blockIdx.x;
   T *pr = p + (size_t)row * ld;
+  const T *p_hi = p + (size_t)(rows - 1) * ld + D;
   const int nv = D >> 2;
   float4 v[LN_MAXV];
   float ss = 0.f;
@@ -444,7 +448,7 @@ rmsnorm_rope_kernel(T *__restrict__ p, int ld, int D, int head_dim,
         u = make_float4(u.x * a.x - u.y * a.y, u.x * a.y + u.y * a.x,
                         u.z * b.x - u.w * b.y, u.z * b.y + u.w * b.x);
       }
-      store4(pr + 4 * c, u);
+      if (WAN_DBG_OK(pr + 4 * c, 4 * sizeof(T), p, p_hi, dbg, WAN_DBG_CODE_BASE + 6)) store4(pr + 4 * c, u);
     }
   }
 }
@@ -454,10 +458,10 @@ static int launch_rr(void *p, int dtype, int rows, int ld, int D, int head_dim, 
                      float eps, const float *rope, int L, int H, int W, int tok0, cudaStream_t s) {
   if (dtype == WAN_BF16)
     rmsnorm_rope_kernel<__nv_bfloat16, NORM, ROPE><<<rows, LN_THREADS, 0, s>>>(
-        (__nv_bfloat16 *)p, ld, D, head_dim, gain, eps, rope, L, H, W, tok0);
+        (__nv_bfloat16 *)p, ld, D, head_dim, gain, eps, rope, L, H, W, tok0, rows, dbg_word());
   else
     rmsnorm_rope_kernel<float, NORM, ROPE><<<rows, LN_THREADS, 0, s>>>(
-        (float *)p, ld, D, head_dim, gain, eps, rope, L, H, W, tok0);
+        (float *)p, ld, D, head_dim, gain, eps, rope, L, H, W, tok0, rows, dbg_word());
   WAN_CHECK_LAUNCH("rmsnorm_rope");
   return WAN_OK;
 }
@@ -496,7 +500,7 @@ struct PermuteArgs {
 };
 
 __global__ void permute_chunks_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, PermuteArgs a,
-                                      long long vpc, long long total) {
+                                      long long vpc, long long total, int *dbg) {
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const long long chunk = i / vpc, v = i - chunk * vpc;
@@ -506,7 +510,7 @@ __global__ void permute_chunks_kernel(const uint4 *__restrict__ src, uint4 *__re
       rem /= a.dst_ext[k];
       off += j * a.src_stride[k];
     }
-    dst[i] = src[off * vpc + v];
+    if (WAN_DBG_OK(dst + i, 16, dst, dst + total, dbg, WAN_DBG_CODE_BASE + 7)) dst[i] = src[off * vpc + v];
   }
 }
 
@@ -528,7 +532,7 @@ int launch_permute_chunks(const void *src, void *dst, int nd, const int *dims, c
   const long long want = (total + 255) / 256;
   const int blocks = (int)(want < 148LL * 16 ? want : 148LL * 16);
   permute_chunks_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4 *>(src), static_cast<uint4 *>(dst), a,
-                                               vpc, total);
+                                               vpc, total, dbg_word());
   WAN_CHECK_LAUNCH("permute_chunks");
   return WAN_OK;
 }
@@ -540,7 +544,8 @@ int launch_permute_chunks(const void *src, void *dst, int nd, const int *dims, c
 // ----------------------------------------------------------------------------
 __global__ void scale_rows_kernel(__nv_bfloat16 *__restrict__ p, int rows, int ld, int D,
                                   const float *__restrict__ ss, int ss_stride, int parts, float inv_d,
-                                  float eps) {
+                                  float eps, int *dbg) {
+  const __nv_bfloat16 *p_hi = p + (size_t)(rows - 1) * ld + D;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -557,7 +562,7 @@ __global__ void scale_rows_kernel(__nv_bfloat16 *__restrict__ p, int rows, int l
       h = __floats2bfloat162_rn(f.x * r, f.y * r);
       w[e] = *reinterpret_cast<uint32_t *>(&h);
     }
-    pr[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    if (WAN_DBG_OK(pr + c, 16, p, p_hi, dbg, WAN_DBG_CODE_BASE + 8)) pr[c] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -567,7 +572,7 @@ int launch_scale_rows(void *p, int rows, int ld, int D, const float *ss, int ss_
   if (D % 8 || ld % 8 || parts < 1 || parts > 32) return set_error(WAN_EUNSUPPORTED, "scale_rows: D=%d", D);
   const int warps = 8;
   scale_rows_kernel<<<(rows + warps - 1) / warps, warps * 32, 0, s>>>(
-      static_cast<__nv_bfloat16 *>(p), rows, ld, D, ss, ss_stride, parts, 1.0f / (float)D, eps);
+      static_cast<__nv_bfloat16 *>(p), rows, ld, D, ss, ss_stride, parts, 1.0f / (float)D, eps, dbg_word());
   WAN_CHECK_LAUNCH("scale_rows");
   return WAN_OK;
 }
@@ -603,7 +608,7 @@ int launch_rope_table(int head_dim, int max_pos, double theta, float *table, cud
 // ----------------------------------------------------------------------------
 template <typename VT, bool CFG>
 __global__ void euler_cfg_kernel(float *__restrict__ x, const VT *__restrict__ vc,
-                                 const VT *__restrict__ vu, size_t n, float scale, float dt) {
+                                 const VT *__restrict__ vu, size_t n, float scale, float dt, int *dbg) {
   const size_t nv = n >> 2;
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nv; i += stride) {
@@ -619,7 +624,7 @@ __global__ void euler_cfg_kernel(float *__restrict__ x, const VT *__restrict__ v
     xv.y = fmaf(dt, v.y, xv.y);
     xv.z = fmaf(dt, v.z, xv.z);
     xv.w = fmaf(dt, v.w, xv.w);
-    store4(x + 4 * i, xv);
+    if (WAN_DBG_OK(x + 4 * i, 16, x, x + n, dbg, WAN_DBG_CODE_BASE + 9)) store4(x + 4 * i, xv);
   }
   // ragged tail (n % 4 elements)
   const size_t t = 4 * nv + blockIdx.x * (size_t)blockDim.x + threadIdx.x;
@@ -630,7 +635,7 @@ __global__ void euler_cfg_kernel(float *__restrict__ x, const VT *__restrict__ v
       const float u = ElemIO<VT>::load(vu + t);
       v = fmaf(scale, c - u, u);
     }
-    x[t] = fmaf(dt, v, x[t]);
+    if (WAN_DBG_OK(x + t, 4, x, x + n, dbg, WAN_DBG_CODE_BASE + 9)) x[t] = fmaf(dt, v, x[t]);
   }
 }
 
@@ -641,9 +646,9 @@ static void euler_launch(float *x, const void *vc, const void *vu, size_t n, flo
   int blocks = (int)((nv + 255) / 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
   if (vu)
-    euler_cfg_kernel<VT, true><<<blocks, 256, 0, s>>>(x, (const VT *)vc, (const VT *)vu, n, scale, dt);
+    euler_cfg_kernel<VT, true><<<blocks, 256, 0, s>>>(x, (const VT *)vc, (const VT *)vu, n, scale, dt, dbg_word());
   else
-    euler_cfg_kernel<VT, false><<<blocks, 256, 0, s>>>(x, (const VT *)vc, nullptr, n, scale, dt);
+    euler_cfg_kernel<VT, false><<<blocks, 256, 0, s>>>(x, (const VT *)vc, nullptr, n, scale, dt, dbg_word());
 }
 
 int launch_euler_cfg(float *x, const void *vc, const void *vu, int vdt, size_t n, float scale,

@@ -102,12 +102,16 @@ __global__ void __launch_bounds__(THREADS) gemm_simt_kernel(const GemmArgs g) {
         xv.y = fmaf(gv.y, v[j + 1], xv.y);
         xv.z = fmaf(gv.z, v[j + 2], xv.z);
         xv.w = fmaf(gv.w, v[j + 3], xv.w);
-        store4(xr + j, xv);
+        if (WAN_DBG_OK(xr + j, 16, g.X, g.X + (size_t)(g.M - 1) * g.ldx + g.N, g.dbg, WAN_DBG_CODE_BASE + 10))
+          store4(xr + j, xv);
       }
     } else {
       T *cr = static_cast<T *>(g.C) + (size_t)m * g.ldc + nb;
-      store4(cr, make_float4(v[0], v[1], v[2], v[3]));
-      store4(cr + 4, make_float4(v[4], v[5], v[6], v[7]));
+      const T *c_hi = static_cast<const T *>(g.C) + (size_t)(g.M - 1) * g.ldc + g.N;
+      if (WAN_DBG_OK(cr, 8 * sizeof(T), g.C, c_hi, g.dbg, WAN_DBG_CODE_BASE + 11)) {
+        store4(cr, make_float4(v[0], v[1], v[2], v[3]));
+        store4(cr + 4, make_float4(v[4], v[5], v[6], v[7]));
+      }
     }
   }
 }
@@ -132,7 +136,9 @@ int gemm_simt(const GemmArgs &g, int dtype, cudaStream_t s) {
     return set_error(WAN_EUNSUPPORTED, "gemm_simt: M=%d N=%d K=%d", g.M, g.N, g.K);
   if (g.M == 0 || g.N == 0) return WAN_OK;
   if ((g.M + BM - 1) / BM > 65535) return set_error(WAN_EINVAL, "gemm_simt: M too large");
-  return dtype == WAN_BF16 ? launch_t<__nv_bfloat16>(g, s) : launch_t<float>(g, s);
+  GemmArgs gd = g;
+  if (!gd.dbg) gd.dbg = dbg_word();
+  return dtype == WAN_BF16 ? launch_t<__nv_bfloat16>(gd, s) : launch_t<float>(gd, s);
 }
 
 }  // namespace wan

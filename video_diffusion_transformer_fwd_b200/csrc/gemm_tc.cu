@@ -6,24 +6,32 @@
 // same 128 bytes), and the epilogue multiplies the accumulator by
 // a_scale[m] * b_scale before the bias.
 //
-// Persistent kernel on CTA pairs (clusters of 2, one CTA per SM): each pair
-// computes 256 x 256 output tiles with tcgen05.mma.cta_group::2 (M = 256 split
-// 128/128 across the two CTAs' TMEM, N = 256, K = 16), K in steps of 64:
+// Persistent kernel on CTA pairs (clusters of 2, one CTA per SM) with
+// tcgen05.mma.cta_group::2 (M = 256 split 128/128 across the two CTAs' TMEM,
+// N = 256 per instruction, K = 16), K in steps of 64, in two tile widths:
+//   wide   256 x 512 output tiles (two N = 256 products per K step sharing
+//          the A stage): per CTA a stage holds 128 rows of A and 256 rows
+//          of B (48 KB), 4 stages; one 512-column TMEM accumulator; 8
+//          epilogue warps. A is read once per 512 output columns, so the
+//          operand traffic from L2 per flop is 3/4 of the narrow tile's.
+//   narrow 256 x 256 tiles, 32 KB stages, 6 stages, two 256-column TMEM
+//          accumulators (the epilogue of one tile overlaps the next
+//          tile's products), 4 epilogue warps; used when a weight segment
+//          is not a multiple of 512 columns.
+// Warp roles:
 //   warp 0      TMA producer in both CTAs: this CTA's 128 rows of A and its
-//               half (128 rows) of B per stage into a 6-stage ring
-//               (128-byte swizzle); bytes of both CTAs are counted on the
-//               leader CTA's "full" barrier;
-//   warp 1      MMA issuer (leader CTA only): 4 pair MMAs per stage into one
-//               of two TMEM accumulators (2 x 256 fp32 columns per CTA);
-//               commits free the stage in both CTAs and publish the
-//               accumulator to both CTAs' epilogues;
-//   warps 2..5  epilogue in both CTAs: tcgen05.ld of this CTA's 128 rows
-//               (warp w reads TMEM lanes 32*(w%4)..+31), bias, GELU or gated
-//               residual, stores to global (the residual add x += g*y goes
-//               through a swizzled smem tile and a TMA reduce-add into x,
-//               or a TMA store when x is written rather than accumulated);
-//               then a release arrive on the leader's "accumulator empty"
-//               barrier.
+//               half of B per stage (128-byte swizzle); bytes of both CTAs
+//               are counted on the leader CTA's "full" barrier;
+//   warp 1      MMA issuer (leader CTA only); commits free the stage in both
+//               CTAs and publish the accumulator to both CTAs' epilogues;
+//   warps 2..   epilogue in both CTAs: tcgen05.ld of this CTA's 128 rows
+//               (warp w reads TMEM lanes 32*(w%4)..+31; in the wide tile
+//               warps 2-5 take columns 0-255 and warps 6-9 columns 256-511),
+//               bias, GELU or gated residual, stores to global (the residual
+//               add x += g*y goes through a swizzled smem tile and a TMA
+//               reduce-add into x, or a TMA store when x is written rather
+//               than accumulated); then a release arrive on the leader's
+//               "accumulator empty" barrier.
 // Tiles are walked in groups of 8 M-tiles (2048 rows) so a wave of pairs
 // shares A and B panels in L2. Every wait is bounded (sm100::mbar_wait).
 #include "common.cuh"
@@ -35,21 +43,32 @@ namespace {
 using namespace sm100;
 
 constexpr int BM = 128;                  // rows per CTA (256 per pair)
-constexpr int BN = 256;                  // columns per tile (128 B rows per CTA)
 constexpr int BK = 64;
-constexpr int STAGES = 6;
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
-constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of B
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 192;
 constexpr int GROUP_M = 8;               // pair tiles (256 rows) per raster group
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC = idesc_bf16(2 * BM, BN, 0);
-constexpr uint32_t IDESC8 = idesc_e4m3(2 * BM, BN);
+constexpr uint32_t IDESC = idesc_bf16(2 * BM, 256, 0);
+constexpr uint32_t IDESC8 = idesc_e4m3(2 * BM, 256);
 constexpr int BK8 = 128;                 // e4m3 elements per stage row (128 bytes)
 constexpr int STG_BYTES = 32 * 32 * 4;  // one warp's 32 x 32 fp32 staging tile (128-byte swizzle)
-constexpr int EPI_SMEM = 4 * 2 * STG_BYTES;  // 4 epilogue warps, double-buffered
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_SMEM + 256;
+constexpr bool USE_WIDE = true;          // 256 x 512 tiles wherever the shape allows
+
+// Tile geometry of the two variants.
+template <bool WIDE>
+struct Geo {
+  static constexpr int BN = WIDE ? 512 : 256;              // output columns per pair tile
+  static constexpr int STAGES = WIDE ? 4 : 6;
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;        // this CTA's half of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_WARPS = WIDE ? 8 : 4;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int NACC = WIDE ? 1 : 2;                // TMEM accumulators (BN columns each)
+  static constexpr int NSTG = WIDE ? 1 : 2;                // residual staging tiles per epilogue warp
+  static constexpr int EPI_SMEM = EPI_WARPS * NSTG * STG_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_SMEM + 256;
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+  static_assert(NACC * BN <= (int)TMEM_COLS, "TMEM columns");
+};
 
 struct TcParams {
   int M, N, K, segN;
@@ -64,6 +83,7 @@ struct TcParams {
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
   const float *rope; int rope_mask; int L, H, W; int head_dim; int tok0;   // L: rows per sequence
   int *watchdog;
+  const void *c_hi, *ss_hi; int *dbg;     // debug bounds checks: ends of C and ss
 };
 
 __device__ __forceinline__ void tile_coords(int t, const TcParams &p, int &mb, int &nb) {
@@ -80,17 +100,20 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t lo16) {
   return __uint_as_float(lo16 << 16);
 }
 
-template <int EPI, bool F8>
-__global__ void __launch_bounds__(THREADS, 1)
+template <int EPI, bool F8, bool WIDE>
+__global__ void __launch_bounds__(Geo<WIDE>::THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
                const __grid_constant__ CUtensorMap tmX, const TcParams p) {
+  using G = Geo<WIDE>;
+  constexpr int BN = G::BN, STAGES = G::STAGES, B_BYTES = G::B_BYTES, STAGE_BYTES = G::STAGE_BYTES;
+  constexpr int NACC = G::NACC, NSTG = G::NSTG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
   uint8_t *sB = smem + STAGES * A_BYTES;
   uint8_t *sE = smem + STAGES * STAGE_BYTES;      // epilogue staging (residual epilogue)
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sE + EPI_SMEM);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sE + G::EPI_SMEM);
   uint64_t *full = bars, *empty = bars + STAGES, *tfull = bars + 2 * STAGES, *tempty = bars + 2 * STAGES + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -119,9 +142,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       mbar_init(smem_u32(&tfull[b]), 1);
-      mbar_init(smem_u32(&tempty[b]), 8);
+      mbar_init(smem_u32(&tempty[b]), 2 * G::EPI_WARPS);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -144,7 +167,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int fills[STAGES] = {0, 0, 0, 0, 0, 0};
+      int fills[STAGES];
+#pragma unroll
+      for (int st = 0; st < STAGES; ++st) fills[st] = 0;
       bool ok = true;
       for (int t = pair; t < p.num_tiles && ok; t += npairs) {
         int mb, nb;
@@ -153,7 +178,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const int seg = n0 / p.segN;
         const CUtensorMap *bm = seg == 0 ? &tmB0 : (seg == 1 ? &tmB1 : &tmB2);
         const int a_row = mb * 2 * BM + (int)rank * BM;
-        const int b_row = n0 - seg * p.segN + (int)rank * (BN / 2);
+        const int b_row = n0 - seg * p.segN + (int)rank * 128;   // this CTA's 128 rows of each N = 256 half
         for (int kb = 0; kb < p.num_k; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, p.watchdog, 0x101)) { ok = false; break; }
           const uint32_t fb_local = smem_u32(&full[stage]);
@@ -162,6 +187,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const int kx = kb * (F8 ? BK8 : BK);
           tma_load_2d_pair(smem_u32(sA + stage * A_BYTES), &tmA, kx, a_row, fb);
           tma_load_2d_pair(smem_u32(sB + stage * B_BYTES), bm, kx, b_row, fb);
+          if (WIDE)      // the second N = 256 half of the tile: B rows 256 further
+            tma_load_2d_pair(smem_u32(sB + stage * B_BYTES + B_BYTES / 2), bm, kx, b_row + 256, fb);
           ++fills[stage];
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -183,8 +210,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int i = 0;
       bool ok = true;
       for (int t = pair; t < p.num_tiles && ok; t += npairs, ++i) {
-        const int buf = i & 1;
-        const uint32_t acc_phase = (i >> 1) & 1;
+        const int buf = i % NACC;
+        const uint32_t acc_phase = (i / NACC) & 1;
         if (!mbar_wait(smem_u32(&tempty[buf]), acc_phase ^ 1, abort_flag, p.watchdog, 0x111)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + buf * BN;
@@ -196,11 +223,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           // 4 MMAs of 32 bytes of K per stage (16 bf16 or 32 e4m3 each):
           // the descriptor start address advances 32 bytes (2 in 16-byte units)
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            if (F8)
-              mma_ss_pair_f8(d, a0 + 2 * kk, b0 + 2 * kk, IDESC8, (kb | kk) != 0);
-            else
-              mma_ss_pair(d, a0 + 2 * kk, b0 + 2 * kk, IDESC, (kb | kk) != 0);
+          for (int h = 0; h < BN / 256; ++h) {
+            // N = 256 half h: B rows of this half at + h * B_BYTES / 2, accumulator columns + 256 h
+            const uint64_t bh = b0 + (uint64_t)((h * (B_BYTES / 2)) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              if (F8)
+                mma_ss_pair_f8(d + 256 * h, a0 + 2 * kk, bh + 2 * kk, IDESC8, (kb | kk) != 0);
+              else
+                mma_ss_pair(d + 256 * h, a0 + 2 * kk, bh + 2 * kk, IDESC, (kb | kk) != 0);
+            }
           }
           const uint32_t eb = smem_u32(&empty[stage]);
           tc_commit_pair(eb);
@@ -215,23 +247,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       }
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    // ------------------------------------------------ epilogue (warps 2.., both CTAs)
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int ew = warp - 2;                 // epilogue warp index
+    const int hcol = WIDE ? (ew >> 2) * 256 : 0;   // first tile column of this warp's 256
     const int row = q * 32 + lane;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
-    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[NACC - 1]), 0);
     int stg_count = 0;
     int i = 0;
     for (int t = pair; t < p.num_tiles; t += npairs, ++i) {
       int mb, nb;
       tile_coords(t, p, mb, nb);
-      const int buf = i & 1;
-      const uint32_t acc_phase = (i >> 1) & 1;
+      const int buf = i % NACC;
+      const uint32_t acc_phase = (i / NACC) & 1;
       if (!mbar_wait(smem_u32(&tfull[buf]), acc_phase, abort_flag, p.watchdog, 0x121)) break;
       tc_fence_after();
       const int m = mb * 2 * BM + (int)rank * BM + row;
-      const int n0 = nb * BN;
-      const int seg = n0 / p.segN;
+      const int n0 = nb * BN + hcol;          // this warp's first column
+      const int seg = (nb * BN) / p.segN;
       const __nv_bfloat16 *bias = static_cast<const __nv_bfloat16 *>(p.bias[seg]);
       const int nn0 = n0 - seg * p.segN;
       float rs = 1.f;                        // FP8: dequantization factor of this row
@@ -251,11 +285,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         wpos = tok % p.W;
       }
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < 8; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + c * 32, r);
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + hcol + c * 32, r);
         tmem_ld_wait();
-        if (c == BN / 32 - 1) {
+        if (c == 7) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
@@ -290,8 +324,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const int m0w = mb * 2 * BM + (int)rank * BM + q * 32;       // warp-uniform
           const float *gr = (p.gate && m < p.M)
                                 ? p.gate + (size_t)(m / p.rows_per_gate) * p.gate_stride + n : nullptr;
-          uint8_t *buf = sE + ((warp - 2) * 2 + (stg_count & 1)) * STG_BYTES;
-          if (lane == 0) bulk_wait_group_read<1>();      // this buffer's previous reduce has read it
+          uint8_t *buf = sE + (ew * NSTG + stg_count % NSTG) * STG_BYTES;
+          if (lane == 0) bulk_wait_group_read<NSTG - 1>();   // this buffer's previous reduce has read it
           __syncwarp();
 #pragma unroll
           for (int j16 = 0; j16 < 8; ++j16) {
@@ -362,13 +396,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             u.y = *reinterpret_cast<uint32_t *>(&h1);
             u.z = *reinterpret_cast<uint32_t *>(&h2);
             u.w = *reinterpret_cast<uint32_t *>(&h3);
-            *reinterpret_cast<uint4 *>(cr + j) = u;
+            if (WAN_DBG_OK(cr + j, 16, p.C, p.c_hi, p.dbg, WAN_DBG_CODE_BASE + 1))
+              *reinterpret_cast<uint4 *>(cr + j) = u;
           }
         }
       }
-      // one partial sum per (row, column tile of the segment): no atomics
-      if (EPI == EPI_QKNORM && ss_col >= 0 && m < p.M)
-        p.ss[(size_t)m * p.ss_stride + ss_col * (p.segN / BN) + nn0 / BN] = sq;
+      // one partial sum per (row, 256-column tile of the segment): no atomics
+      if (EPI == EPI_QKNORM && ss_col >= 0 && m < p.M && n0 < p.N)
+      {
+        float *sp = p.ss + (size_t)m * p.ss_stride + ss_col * (p.segN / 256) + nn0 / 256;
+        if (WAN_DBG_OK(sp, 4, p.ss, p.ss_hi, p.dbg, WAN_DBG_CODE_BASE + 2)) *sp = sq;
+      }
     }
   }
 
@@ -380,24 +418,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 1) tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
-template <int EPI, bool F8>
+template <int EPI, bool F8, bool WIDE>
 int launch(const CUtensorMap &ta, const CUtensorMap *tb, const CUtensorMap &tx, const TcParams &p,
            cudaStream_t s) {
+  using G = Geo<WIDE>;
   static int max_pairs = 0;         // per process; the attribute is per function
   if (!max_pairs) {
-    WAN_TRY_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
-                 "gemm_tc smem attribute");
+    WAN_TRY_CUDA(cudaFuncSetAttribute(gemm_tc_kernel<EPI, F8, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      G::SMEM_BYTES), "gemm_tc smem attribute");
     cudaLaunchConfig_t qc = {};
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeClusterDimension;
     qa[0].val.clusterDim.x = 2; qa[0].val.clusterDim.y = 1; qa[0].val.clusterDim.z = 1;
     qc.gridDim = dim3(2 * 74, 1, 1);
-    qc.blockDim = dim3(THREADS, 1, 1);
-    qc.dynamicSmemBytes = SMEM_BYTES;
+    qc.blockDim = dim3(G::THREADS, 1, 1);
+    qc.dynamicSmemBytes = G::SMEM_BYTES;
     qc.attrs = qa;
     qc.numAttrs = 1;
     int clusters = 0;
-    WAN_TRY_CUDA(cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<EPI, F8>, &qc), "gemm_tc occupancy");
+    WAN_TRY_CUDA(cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<EPI, F8, WIDE>, &qc), "gemm_tc occupancy");
     max_pairs = clusters > 0 ? clusters : sm_count() / 2;
   }
   const int pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
@@ -406,13 +445,25 @@ int launch(const CUtensorMap &ta, const CUtensorMap *tb, const CUtensorMap &tx, 
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2; attr[0].val.clusterDim.y = 1; attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.blockDim = dim3(G::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = G::SMEM_BYTES;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  WAN_TRY_CUDA(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI, F8>, ta, tb[0], tb[1], tb[2], tx, p), "gemm_tc launch");
+  WAN_TRY_CUDA(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI, F8, WIDE>, ta, tb[0], tb[1], tb[2], tx, p),
+               "gemm_tc launch");
   return WAN_OK;
+}
+
+template <bool F8, bool WIDE>
+int launch_epi(int epi, const CUtensorMap &ta, const CUtensorMap *tb, const CUtensorMap &tx, const TcParams &p,
+               cudaStream_t s) {
+  switch (epi) {
+    case EPI_STORE: return launch<EPI_STORE, F8, WIDE>(ta, tb, tx, p, s);
+    case EPI_GELU: return launch<EPI_GELU, F8, WIDE>(ta, tb, tx, p, s);
+    case EPI_QKNORM: return launch<EPI_QKNORM, F8, WIDE>(ta, tb, tx, p, s);
+    default: return launch<EPI_RESID, F8, WIDE>(ta, tb, tx, p, s);
+  }
 }
 }  // namespace
 
@@ -426,7 +477,7 @@ bool gemm_tc_supported(const GemmArgs &g) {
       if (!g.b_scale[i]) return false;
   }
   if (g.nseg < 1 || g.nseg > 3 || g.segN * g.nseg != g.N) return false;
-  if (g.nseg > 1 && g.segN % BN) return false;
+  if (g.nseg > 1 && g.segN % 256) return false;
   if (g.lda % 8) return false;
   if (g.epi != EPI_RESID && g.ldc % 8) return false;
   if (g.epi == EPI_RESID && (g.ldx % 4 || !aligned16(g.X) || (g.gate && g.gate_stride % 4))) return false;
@@ -437,7 +488,7 @@ bool gemm_tc_supported(const GemmArgs &g) {
       if (g.gamma[i] && !aligned16(g.gamma[i])) return false;
     }
     if (g.rope && (g.head_dim % 32 || g.segN % g.head_dim)) return false;
-    if (g.segN % BN) return false;             // whole column tiles per segment (partial sums)
+    if (g.segN % 256) return false;            // whole 256-column tiles per segment (partial sums)
   }
   for (int i = 0; i < g.nseg; ++i)
     if (!aligned16(g.Bseg[i]) || (g.bias[i] && !aligned16(g.bias[i]))) return false;
@@ -452,14 +503,17 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   if (rc) return rc;
   for (int i = 0; i < 3; ++i) {
     const int si = i < g.nseg ? i : 0;
-    rc = g.fp8 ? encode_tmap_2d_u8(&tb[i], g.Bseg[si], g.K, g.segN, (uint64_t)g.K, BK8, BN / 2)
-               : encode_tmap_2d_bf16(&tb[i], g.Bseg[si], g.K, g.segN, (uint64_t)g.K * 2, BK, BN / 2);
+    rc = g.fp8 ? encode_tmap_2d_u8(&tb[i], g.Bseg[si], g.K, g.segN, (uint64_t)g.K, BK8, 128)
+               : encode_tmap_2d_bf16(&tb[i], g.Bseg[si], g.K, g.segN, (uint64_t)g.K * 2, BK, 128);
     if (rc) return rc;
   }
   TcParams p = {};
   p.M = g.M; p.N = g.N; p.K = g.K; p.segN = g.segN;
+  // the wide tile when no 512-column tile straddles two weight segments
+  const bool wide = USE_WIDE && (g.nseg == 1 || g.segN % 512 == 0);
+  const int bn = wide ? 512 : 256;
   p.num_m = (g.M + 2 * BM - 1) / (2 * BM);
-  p.num_n = (g.N + BN - 1) / BN;
+  p.num_n = (g.N + bn - 1) / bn;
   p.num_tiles = p.num_m * p.num_n;
   p.num_k = g.K / (g.fp8 ? BK8 : BK);
   p.a_scale = g.a_scale;
@@ -480,22 +534,13 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   p.tok0 = g.tok0;
   p.head_dim = g.head_dim > 0 ? g.head_dim : 128;
   p.watchdog = watchdog_ptr();
+  p.dbg = g.dbg ? g.dbg : dbg_word();
+  if (g.C) p.c_hi = static_cast<const char *>(g.C) + ((size_t)(g.M - 1) * g.ldc + g.N) * 2;
+  if (g.ss) p.ss_hi = g.ss + (size_t)g.M * g.ss_stride;
   CUtensorMap tx = ta;
   if (g.epi == EPI_RESID && (rc = encode_tmap_2d_f32(&tx, g.X, g.N, g.M, (uint64_t)g.ldx * 4, 32, 32))) return rc;
-  if (g.fp8) {
-    switch (g.epi) {
-      case EPI_STORE: return launch<EPI_STORE, true>(ta, tb, tx, p, s);
-      case EPI_GELU: return launch<EPI_GELU, true>(ta, tb, tx, p, s);
-      case EPI_QKNORM: return launch<EPI_QKNORM, true>(ta, tb, tx, p, s);
-      default: return launch<EPI_RESID, true>(ta, tb, tx, p, s);
-    }
-  }
-  switch (g.epi) {
-    case EPI_STORE: return launch<EPI_STORE, false>(ta, tb, tx, p, s);
-    case EPI_GELU: return launch<EPI_GELU, false>(ta, tb, tx, p, s);
-    case EPI_QKNORM: return launch<EPI_QKNORM, false>(ta, tb, tx, p, s);
-    default: return launch<EPI_RESID, false>(ta, tb, tx, p, s);
-  }
+  if (g.fp8) return wide ? launch_epi<true, true>(g.epi, ta, tb, tx, p, s) : launch_epi<true, false>(g.epi, ta, tb, tx, p, s);
+  return wide ? launch_epi<false, true>(g.epi, ta, tb, tx, p, s) : launch_epi<false, false>(g.epi, ta, tb, tx, p, s);
 }
 
 }  // namespace wan

@@ -14,7 +14,7 @@ import os
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libwan.so")
 
-WAN_OK, WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED, WAN_ECUDA, WAN_ETIMEOUT = 0, -1, -2, -3, -4, -5
+WAN_OK, WAN_EINVAL, WAN_EALIGN, WAN_EUNSUPPORTED, WAN_ECUDA, WAN_ETIMEOUT, WAN_EBOUNDS = 0, -1, -2, -3, -4, -5, -6
 WAN_F32, WAN_BF16, WAN_FP8, WAN_FP8_ATTN = 0, 1, 2, 3
 WAN_NOALLOC_WORKSPACE_BYTES = 16 << 20
 (WAN_WS_ACT, WAN_WS_QKV, WAN_WS_O, WAN_WS_QC, WAN_WS_KVC, WAN_WS_OC, WAN_WS_H, WAN_WS_MOD,
@@ -25,7 +25,7 @@ WAN_K_COUNT = 12
 KERNEL_CLASS_NAMES = ("gemm_tc", "gemm_simt", "attn_self", "attn_cross", "attn_simt", "layernorm",
                       "qknorm_rope", "euler_cfg", "misc", "attn_tc", "model", "quant")
 STATUS_NAMES = {0: "WAN_OK", -1: "WAN_EINVAL", -2: "WAN_EALIGN", -3: "WAN_EUNSUPPORTED",
-                -4: "WAN_ECUDA", -5: "WAN_ETIMEOUT"}
+                -4: "WAN_ECUDA", -5: "WAN_ETIMEOUT", -6: "WAN_EBOUNDS"}
 
 
 class WanError(RuntimeError):
@@ -92,6 +92,7 @@ _SIGS = {
     "wan_euler_cfg_step": (_c_int, [_vp, _vp, _vp, _c_int, _sz, ctypes.c_float, ctypes.c_float,
                                     ctypes.c_float, _vp]),
     "wan_device_status": (_c_int, [_vp]),
+    "wan_debug_bounds": (_c_int, []),
     "wan_profile_enable": (_c_int, [_c_int]),
     "wan_selftest_watchdog": (_c_int, [_vp]),
     "wan_profile_read": (_c_int, [_c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]),
@@ -114,11 +115,14 @@ _SIGS = {
 _lib = None
 
 
-def load(path: str = LIB_PATH):
-    """Load libwan.so (raises if it is missing: there is no fallback)."""
+def load(path: str | None = None):
+    """Load libwan.so (raises if it is missing: there is no fallback). The
+    environment variable WAN_LIBRARY may name another build of the library
+    (the debug build, ``build_lib.build(debug=True)``)."""
     global _lib
     if _lib is not None:
         return _lib
+    path = path or os.environ.get("WAN_LIBRARY") or LIB_PATH
     if not os.path.exists(path):
         raise RuntimeError(f"libwan.so not built at {path}; run "
                            "`python -m video_diffusion_transformer_fwd_b200.build_lib`")
@@ -238,6 +242,10 @@ def wan_unipc_step(x, last, m_out, m_prev1, m_prev2, v_cond, v_uncond, v_dtype, 
                    stream):
     return load().wan_unipc_step(x, last, m_out, m_prev1, m_prev2, v_cond, v_uncond, v_dtype, n, guide_scale,
                                  sigma, coef, stream)
+
+
+def wan_debug_bounds():
+    return load().wan_debug_bounds()
 
 
 def wan_device_status(stream):
