@@ -39,9 +39,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # same kernel source (sha256 prefix below); reported as null once the source
 # has changed since the capture.
 TRAFFIC = {
-    # profiles/attn_tc_B1_L16384.md: 652.7 MB per launch at B=1, L=16384, scaled by the
+    # profiles/attn_tc_B1_L16384.md: 652.6 MB per launch at B=1, L=16384, scaled by the
     # query/key rows (x4) to the step's launch at B=2, L=32760
-    "attn_self": {"bytes_per_launch": 4 * 652.7e6, "source_sha": "2028616860a240aa"},
+    "attn_self": {"bytes_per_launch": 4 * 652.6e6, "source_sha": "f80a182236bf1ae4"},
 }
 
 
@@ -356,7 +356,8 @@ def per_config_rows(dev, peaks, iters=5, warmup=2):
     for name, B in PER_CONFIG:
         cfg = dataclasses.replace(configs.get(name), batch=B, blocks=1)
         dims = wan.dims_of(cfg)
-        w = wan.make_weights(synth.block_weights(cfg.dim, cfg.ffn_dim, cfg.dtype, dev, 0))
+        wt = synth.block_weights(cfg.dim, cfg.ffn_dim, cfg.dtype, dev, 0)    # the tensors stay alive
+        w = wan.make_weights(wt)
         acts = synth.block_activations(B, cfg.L, cfg.dim, cfg.text_len, cfg.dtype, dev, 100)
         rope = wan.rope_freqs(cfg.head_dim, 1024, cfg.theta, device=dev)
         ws = wan.alloc_workspace(dims, B, device=dev)
@@ -389,7 +390,7 @@ def per_config_rows(dev, peaks, iters=5, warmup=2):
             "gemm_frac_of_measured_burst": None if g_tf is None else g_tf / burst,
             "kernel_ms": {k: v[1] / iters for k, v in prof.items() if v[0]},
             "clocks": {"sm_mhz": ck.get("sm_mhz"), "reasons": ck.get("reasons")}})
-        del w, acts, ws
+        del w, wt, acts, ws
         torch.cuda.empty_cache()
     return rows
 

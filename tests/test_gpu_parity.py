@@ -198,6 +198,36 @@ def test_tiny_stack_of_40_blocks_and_step():
     assert np.abs(np64(st.x) - ref).max() <= F32_MAX_ABS
 
 
+def test_bf16_stack_of_40_blocks_and_step():
+    """The denoising-step launch sequence at a bf16 size where the whole fp64
+    chain is affordable (40 blocks, dim 512, 4 heads of 128, ffn 1024, grid
+    4 x 8 x 16 = 512 tokens, text 64, CFG pair): the two block-stack outputs
+    (their accumulated change over the 40 blocks) and the CFG-Euler update,
+    every row, against the oracle run block by block on its own outputs."""
+    from video_diffusion_transformer_fwd_b200.step import DenoiseStep
+    cfg = BlockConfig("bf16-chain", 4, 8, 16, 512, 4, 1024, 64, "bf16", batch=2, blocks=40)
+    st = DenoiseStep(cfg, seed=0)
+    x0 = np64(st.x)
+    st.step()
+    torch.cuda.synchronize()
+    assert wan.device_status() == wan.WAN_OK
+    grid = (cfg.F, cfg.H, cfg.W)
+    ctx = np.stack([np64(st.ctx[0]), np64(st.ctx[1])])
+    e0 = np.stack([np64(st.e0[0])] * 2)
+    xb = np.stack([x0, x0])
+    for w in st.weights:
+        xb = O.block_forward(xb, ctx, None, e0, weights64(w), cfg.heads, grid, cfg.eps, cfg.theta)
+    ref = O.euler_cfg_step(x0, xb[0], xb[1], cfg.guide_scale, cfg.sigma, cfg.sigma_next)
+    got_v = np64(st.xb)
+    errs = {"stack_delta_cond": rel_l2(got_v[0] - x0, xb[0] - x0),
+            "stack_delta_uncond": rel_l2(got_v[1] - x0, xb[1] - x0),
+            "cfg_direction": rel_l2(got_v[0] - got_v[1], xb[0] - xb[1]),
+            "step_update": rel_l2(np64(st.x) - x0, ref - x0)}
+    print({k: f"{v:.2e}" for k, v in errs.items()})
+    for k, v in errs.items():
+        assert v <= BF16_REL_L2, (k, v)
+
+
 # ------------------------------------------------------------------ block, bf16 (sampled rows)
 
 def _bf16_block_check(cfg, B=1, same=False, seed=0, gain_scale=1.0, ctx_lens=None):

@@ -16,8 +16,10 @@
 //          operand traffic from L2 per flop is 3/4 of the narrow tile's.
 //   narrow 256 x 256 tiles, 32 KB stages, 6 stages, two 256-column TMEM
 //          accumulators (the epilogue of one tile overlaps the next
-//          tile's products), 4 epilogue warps; used when a weight segment
-//          is not a multiple of 512 columns.
+//          tile's products), 4 epilogue warps; used when K < 4096 (there
+//          the wide tile's epilogue, which cannot overlap, costs more than
+//          its saving in operand traffic) or a weight segment is not a
+//          multiple of 512 columns.
 // Warp roles:
 //   warp 0      TMA producer in both CTAs: this CTA's 128 rows of A and its
 //               half of B per stage (128-byte swizzle); bytes of both CTAs
@@ -509,8 +511,12 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   }
   TcParams p = {};
   p.M = g.M; p.N = g.N; p.K = g.K; p.segN = g.segN;
-  // the wide tile when no 512-column tile straddles two weight segments
-  const bool wide = USE_WIDE && (g.nseg == 1 || g.segN % 512 == 0);
+  // the wide tile when no 512-column tile straddles two weight segments and K
+  // is long enough for its epilogue (which does not overlap the next tile's
+  // products) to be a small share of a tile: measured on the workload's
+  // blocks, wide is 7% faster at K = 5120, even at K = 3072, and 9-10%
+  // slower at K = 1536
+  const bool wide = USE_WIDE && g.K >= 4096 && (g.nseg == 1 || g.segN % 512 == 0);
   const int bn = wide ? 512 : 256;
   p.num_m = (g.M + 2 * BM - 1) / (2 * BM);
   p.num_n = (g.N + bn - 1) / bn;
