@@ -98,6 +98,16 @@ __device__ __forceinline__ void tile_coords(int t, const TcParams &p, int &mb, i
   nb = r / gm;
 }
 
+// GELU (tanh form) for a bf16 output: tanh from the hardware approximation
+// (tanh.approx.f32, relative error about 2^-11), below the bf16 rounding of
+// the result (2^-9).
+__device__ __forceinline__ float gelu_tanh_bf16out(float z) {
+  const float k0 = 0.7978845608028654f, k1 = 0.044715f;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(k0 * fmaf(k1 * z, z * z, z)));
+  return 0.5f * z * (1.0f + t);
+}
+
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t lo16) {
   return __uint_as_float(lo16 << 16);
 }
@@ -297,11 +307,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
         }
         const int n = n0 + c * 32;
-        if (EPI == EPI_RESID) {
-          if (mb * 2 * BM + (int)rank * BM + q * 32 >= p.M || n >= p.N) continue;   // warp-uniform
-        } else if (m >= p.M || n >= p.N) {
-          continue;
-        }
+        // warp-uniform: rows of the warp beyond M are clipped by the tensor map
+        if (mb * 2 * BM + (int)rank * BM + q * 32 >= p.M || n >= p.N) continue;
         float v[32];
         const uint4 *bp = reinterpret_cast<const uint4 *>(bias + nn0 + c * 32);
 #pragma unroll
@@ -383,12 +390,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               }
             }
           }
-          __nv_bfloat16 *cr = static_cast<__nv_bfloat16 *>(p.C) + (size_t)m * p.ldc + n;
+          // bf16 rows of two consecutive 32-column chunks go through a swizzled
+          // 32 x 64 shared-memory tile (128-byte rows, 16-byte chunk k of row r
+          // at k ^ (r & 7)) and one TMA store of the tile
+          const int sub = c & 1;
+          const int m0w = mb * 2 * BM + (int)rank * BM + q * 32;       // warp-uniform
+          uint8_t *sbuf = sE + (ew * NSTG + stg_count % NSTG) * STG_BYTES;
+          if (sub == 0) {
+            if (lane == 0) bulk_wait_group_read<NSTG - 1>();   // this tile's previous store has read it
+            __syncwarp();
+          }
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
             float a[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a[e] = (EPI == EPI_GELU) ? gelu_tanh(v[j + e]) : v[j + e];
+            for (int e = 0; e < 8; ++e) a[e] = (EPI == EPI_GELU) ? gelu_tanh_bf16out(v[j + e]) : v[j + e];
             __nv_bfloat162 h0 = __floats2bfloat162_rn(a[0], a[1]);
             __nv_bfloat162 h1 = __floats2bfloat162_rn(a[2], a[3]);
             __nv_bfloat162 h2 = __floats2bfloat162_rn(a[4], a[5]);
@@ -398,8 +414,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             u.y = *reinterpret_cast<uint32_t *>(&h1);
             u.z = *reinterpret_cast<uint32_t *>(&h2);
             u.w = *reinterpret_cast<uint32_t *>(&h3);
-            if (WAN_DBG_OK(cr + j, 16, p.C, p.c_hi, p.dbg, WAN_DBG_CODE_BASE + 1))
-              *reinterpret_cast<uint4 *>(cr + j) = u;
+            const int k = sub * 4 + (j >> 3);
+            *reinterpret_cast<uint4 *>(sbuf + lane * 128 + ((k ^ (lane & 7)) << 4)) = u;
+          }
+          if (sub == 1) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmX, smem_u32(sbuf), n - 32, m0w);
+              bulk_commit_group();
+            }
+            ++stg_count;
           }
         }
       }
@@ -412,7 +437,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
   }
 
-  if (EPI == EPI_RESID && warp >= 2 && lane == 0) bulk_wait_group_all();   // reduces done with smem
+  if (warp >= 2 && lane == 0) bulk_wait_group_all();   // this warp's TMA stores / reduces are done
 
   tc_fence_before();
   cluster_sync_all();               // the peer's smem and TMEM stay live until the leader is done
@@ -481,7 +506,7 @@ bool gemm_tc_supported(const GemmArgs &g) {
   if (g.nseg < 1 || g.nseg > 3 || g.segN * g.nseg != g.N) return false;
   if (g.nseg > 1 && g.segN % 256) return false;
   if (g.lda % 8) return false;
-  if (g.epi != EPI_RESID && g.ldc % 8) return false;
+  if (g.epi != EPI_RESID && (g.ldc % 8 || g.N % 64 || !aligned16(g.C))) return false;   // staged 64-column TMA stores
   if (g.epi == EPI_RESID && (g.ldx % 4 || !aligned16(g.X) || (g.gate && g.gate_stride % 4))) return false;
   if (g.gate_bias && !aligned16(g.gate_bias)) return false;
   if (g.epi == EPI_QKNORM) {
@@ -543,8 +568,13 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   p.dbg = g.dbg ? g.dbg : dbg_word();
   if (g.C) p.c_hi = static_cast<const char *>(g.C) + ((size_t)(g.M - 1) * g.ldc + g.N) * 2;
   if (g.ss) p.ss_hi = g.ss + (size_t)g.M * g.ss_stride;
+  // the epilogue's store target: x (fp32, 32 x 32 boxes) for the residual, else C (bf16, 64 x 32 boxes)
   CUtensorMap tx = ta;
-  if (g.epi == EPI_RESID && (rc = encode_tmap_2d_f32(&tx, g.X, g.N, g.M, (uint64_t)g.ldx * 4, 32, 32))) return rc;
+  if (g.epi == EPI_RESID) {
+    if ((rc = encode_tmap_2d_f32(&tx, g.X, g.N, g.M, (uint64_t)g.ldx * 4, 32, 32))) return rc;
+  } else if ((rc = encode_tmap_2d_bf16(&tx, g.C, g.N, g.M, (uint64_t)g.ldc * 2, 64, 32))) {
+    return rc;
+  }
   if (g.fp8) return wide ? launch_epi<true, true>(g.epi, ta, tb, tx, p, s) : launch_epi<true, false>(g.epi, ta, tb, tx, p, s);
   return wide ? launch_epi<false, true>(g.epi, ta, tb, tx, p, s) : launch_epi<false, false>(g.epi, ta, tb, tx, p, s);
 }
