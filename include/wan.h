@@ -461,10 +461,12 @@ int wan_euler_cfg_step(float *x, const void *v_cond, const void *v_uncond,
 int wan_device_status(wan_stream_t stream);
 
 /* wan_debug_bounds -- 1 in a debug build (compiled with WAN_DEBUG_BOUNDS:
- * every plain global store of the block's kernels -- the GEMM and attention
- * epilogues, LayerNorm, RMSNorm / RoPE, the k / q row scaling, the chunk
- * permutation, CFG-Euler -- is checked against its buffer's extent before
- * it is made), 0 otherwise. */
+ * every plain global store of the block's kernels -- the GEMM epilogue's
+ * q / k sums of squares, LayerNorm, RMSNorm / RoPE, the k / q row scaling,
+ * the chunk permutation, CFG-Euler, the CUDA-core GEMM and attention -- is
+ * checked against its buffer's extent before it is made; the tensor-core
+ * GEMM and attention write their outputs with TMA stores and reduce-adds,
+ * which the tensor maps clip), 0 otherwise. */
 int wan_debug_bounds(void);
 
 /* wan_selftest_watchdog -- enqueue a one-CTA kernel whose bounded wait on an

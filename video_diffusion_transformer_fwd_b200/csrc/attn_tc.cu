@@ -19,8 +19,12 @@
 //               (K_{j+2} as soon as S(j) is done) and V tiles into one slot
 //               (V_{j+1} once PV(j) is done), 32 KB each (128-byte swizzle).
 // TMEM: S_0 | S_1 | O_0 | O_1, 128 fp32 columns each (512 total).
+// At the end each softmax thread writes its row of O / l (bf16) into its
+// tile's P buffer, in the same swizzled layout, and one thread per tile
+// stores the tile with two TMA stores.
 // Every wait is bounded (sm100::mbar_wait); keys at or beyond the sequence's
-// key length are masked; rows of a tile beyond Lq are computed but not stored.
+// key length are masked; rows of a tile beyond Lq are computed but clipped by
+// the output's tensor map.
 #include "common.cuh"
 #include "sm100.cuh"
 
@@ -49,7 +53,6 @@ struct FaParams {
   __nv_bfloat16 *o; int ldo;
   const float *q_ss; int q_ss_stride; int q_ss_parts; float q_ss_inv_n; float q_ss_eps;   // optional per-row RMS factor of q
   int *watchdog;
-  const void *o_hi; int *dbg;           // debug bounds checks: end of o
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -87,13 +90,21 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// 3D tiled store from shared memory (x inner, y row, z batch); rows and
+// columns beyond the tensor are clipped
+__device__ __forceinline__ void tma_store_3d(const void *tmap, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(src), "r"(x), "r"(y), "r"(z) : "memory");
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, const FaParams p) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               const FaParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = smem;                               // 2 tiles
@@ -354,8 +365,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       ok = mbar_wait(smem_u32(&pv_done[i]), (nkt - 1) & 1, abort_flag, p.watchdog, 0x223);
       tc_fence_after();
     }
+    // O / l as bf16 into the P_i tile (free once PV_i of the last key tile is
+    // done; the same swizzled layout, two boxes of 64 columns), then one
+    // thread of the tile writes it with two TMA stores (rows beyond Lq are
+    // clipped by the tensor map)
     const float inv = (l > 0.f) ? 1.0f / l : 0.f;
-    __nv_bfloat16 *orow = p.o + (size_t)(b * p.Lq + (row < p.Lq ? row : 0)) * p.ldo + h * D;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       uint32_t o[32];
@@ -366,18 +380,23 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[e] = 0u;
       }
-      if (row < p.Lq && ok) {
-        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint4 u;
-          u.x = pack_bf16(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv);
-          u.y = pack_bf16(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv);
-          u.z = pack_bf16(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv);
-          u.w = pack_bf16(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv);
-          if (WAN_DBG_OK(dst + e, 16, p.o, p.o_hi, p.dbg, WAN_DBG_CODE_BASE + 3)) dst[e] = u;
-        }
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t k = (uint32_t)(c * 4 + e);                     // 16-byte chunk of the row
+        const uint32_t addr = p_row + (k >> 3) * BOX_BYTES + (((k & 7u) ^ ((uint32_t)r & 7u)) << 4);
+        st_shared_v4(addr, pack_bf16(__uint_as_float(o[8 * e + 0]) * inv, __uint_as_float(o[8 * e + 1]) * inv),
+                     pack_bf16(__uint_as_float(o[8 * e + 2]) * inv, __uint_as_float(o[8 * e + 3]) * inv),
+                     pack_bf16(__uint_as_float(o[8 * e + 4]) * inv, __uint_as_float(o[8 * e + 5]) * inv),
+                     pack_bf16(__uint_as_float(o[8 * e + 6]) * inv, __uint_as_float(o[8 * e + 7]) * inv));
       }
+    }
+    fence_proxy_async_smem();
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + i) : "memory");      // the tile's 4 warps
+    if (qw == 0 && lane == 0 && ok) {
+      for (int half = 0; half < 2; ++half)
+        tma_store_3d(&tmO, smem_u32(sP + i * TILE_BYTES + half * BOX_BYTES), h * D + half * 64, q0 + i * TQ, b);
+      bulk_commit_group();
+      bulk_wait_group_all();
     }
   }
 
@@ -405,6 +424,8 @@ int attention_tc(const AttnArgs &a, cudaStream_t s) {
   if (rc) return rc;
   if ((rc = encode_tmap_3d_bf16(&tk, a.k, inner, Lk, a.B, (uint64_t)a.ldk * 2, (uint64_t)a.Lk * a.ldk * 2 + (a.Lk ? 0 : 16), 64, TK))) return rc;
   if ((rc = encode_tmap_3d_bf16(&tv, a.v, inner, Lk, a.B, (uint64_t)a.ldv * 2, (uint64_t)a.Lk * a.ldv * 2 + (a.Lk ? 0 : 16), 64, TK))) return rc;
+  CUtensorMap to;
+  if ((rc = encode_tmap_3d_bf16(&to, a.o, inner, a.Lq, a.B, (uint64_t)a.ldo * 2, (uint64_t)a.Lq * a.ldo * 2, 64, TQ))) return rc;
   static bool attr_set = false;
   if (!attr_set) {
     WAN_TRY_CUDA(cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
@@ -418,10 +439,8 @@ int attention_tc(const AttnArgs &a, cudaStream_t s) {
   p.q_ss_inv_n = a.q_ss_n > 0.f ? 1.0f / a.q_ss_n : 0.f; p.q_ss_eps = a.q_ss_eps;
   p.o = static_cast<__nv_bfloat16 *>(a.o); p.ldo = a.ldo;
   p.watchdog = watchdog_ptr();
-  p.dbg = a.dbg ? a.dbg : dbg_word();
-  p.o_hi = static_cast<const char *>(a.o) + ((size_t)(a.B * a.Lq - 1) * a.ldo + (size_t)a.heads * D) * 2;
   dim3 grid((a.Lq + 2 * TQ - 1) / (2 * TQ), a.heads, a.B);
-  attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tq, tk, tv, p);
+  attn_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(tq, tk, tv, to, p);
   WAN_CHECK_LAUNCH("attention_tc");
   return WAN_OK;
 }

@@ -85,7 +85,7 @@ struct TcParams {
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
   const float *rope; int rope_mask; int L, H, W; int head_dim; int tok0;   // L: rows per sequence
   int *watchdog;
-  const void *c_hi, *ss_hi; int *dbg;     // debug bounds checks: ends of C and ss
+  const void *ss_hi; int *dbg;            // debug bounds checks: end of ss
 };
 
 __device__ __forceinline__ void tile_coords(int t, const TcParams &p, int &mb, int &nb) {
@@ -566,7 +566,6 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   p.head_dim = g.head_dim > 0 ? g.head_dim : 128;
   p.watchdog = watchdog_ptr();
   p.dbg = g.dbg ? g.dbg : dbg_word();
-  if (g.C) p.c_hi = static_cast<const char *>(g.C) + ((size_t)(g.M - 1) * g.ldc + g.N) * 2;
   if (g.ss) p.ss_hi = g.ss + (size_t)g.M * g.ss_stride;
   // the epilogue's store target: x (fp32, 32 x 32 boxes) for the residual, else C (bf16, 64 x 32 boxes)
   CUtensorMap tx = ta;
