@@ -108,7 +108,6 @@ __global__ void __launch_bounds__(THREADS) attn_simt_kernel(const AttnArgs a) {
   if (!active) return;
   const float inv = (l > 0.f) ? 1.0f / l : 0.f;
   T *orow = static_cast<T *>(a.o) + (size_t)(b * a.Lq + r) * a.ldo + h * D;
-#pragma unroll
   const T *o_hi = static_cast<const T *>(a.o) + (size_t)(a.B * a.Lq - 1) * a.ldo + (size_t)a.heads * D;
 #pragma unroll
   for (int c = 0; c < NC; ++c)

@@ -545,7 +545,6 @@ int launch_permute_chunks(const void *src, void *dst, int nd, const int *dims, c
 __global__ void scale_rows_kernel(__nv_bfloat16 *__restrict__ p, int rows, int ld, int D,
                                   const float *__restrict__ ss, int ss_stride, int parts, float inv_d,
                                   float eps, int *dbg) {
-  const __nv_bfloat16 *p_hi = p + (size_t)(rows - 1) * ld + D;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -562,7 +561,8 @@ __global__ void scale_rows_kernel(__nv_bfloat16 *__restrict__ p, int rows, int l
       h = __floats2bfloat162_rn(f.x * r, f.y * r);
       w[e] = *reinterpret_cast<uint32_t *>(&h);
     }
-    if (WAN_DBG_OK(pr + c, 16, p, p_hi, dbg, WAN_DBG_CODE_BASE + 8)) pr[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    if (WAN_DBG_OK(pr + c, 16, p, p + (size_t)(rows - 1) * ld + D, dbg, WAN_DBG_CODE_BASE + 8))
+      pr[c] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 

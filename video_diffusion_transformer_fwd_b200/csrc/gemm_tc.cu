@@ -83,7 +83,7 @@ struct TcParams {
   const float *a_scale; const float *b_scale[3];      // FP8: per row of A, per weight segment
   // q/k RMSNorm + RoPE epilogue (EPI_QKNORM)
   const float *gamma[3]; float *ss; int ss_stride; int ss_col[3];
-  const float *rope; int rope_mask; int L, H, W; int head_dim; int tok0;   // L: rows per sequence
+  const float *rope; int rope_mask; int rope_vec; int L, H, W; int head_dim; int tok0;   // L: rows per sequence
   int *watchdog;
   const void *ss_hi; int *dbg;            // debug bounds checks: end of ss
 };
@@ -273,8 +273,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       tile_coords(t, p, mb, nb);
       const int buf = i % NACC;
       const uint32_t acc_phase = (i / NACC) & 1;
-      if (!mbar_wait(smem_u32(&tfull[buf]), acc_phase, abort_flag, p.watchdog, 0x121)) break;
-      tc_fence_after();
       const int m = mb * 2 * BM + (int)rank * BM + row;
       const int n0 = nb * BN + hcol;          // this warp's first column
       const int seg = (nb * BN) / p.segN;
@@ -296,6 +294,29 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         hpos = (tok / p.W) % p.H;
         wpos = tok % p.W;
       }
+      // the bias, gamma, gate and RoPE-table lines this warp reads go to L1
+      // while the tile's products still run (each would otherwise cost its
+      // chunk an L2 round trip)
+      if (n0 < p.N) {
+        const int last = min(255, p.N - n0 - 1);      // the warp's last column that exists
+        if (bias && lane < 5) prefetch_l1(bias + nn0 + min(lane < 4 ? lane * 64 : 255, last));
+        const float *pf = nullptr;
+        if (EPI == EPI_QKNORM) pf = gam ? gam + nn0 : nullptr;
+        if (EPI == EPI_RESID && p.gate && p.rows_per_gate > 1 && m < p.M)
+          pf = p.gate + (size_t)(m / p.rows_per_gate) * p.gate_stride + n0;
+        if (pf && lane >= 8 && lane < 17) prefetch_l1(pf + min(lane < 16 ? (lane - 8) * 32 : 255, last));
+        if (EPI == EPI_QKNORM && do_rope && p.head_dim == 128) {
+          // one table row is 64 pairs (512 bytes): t pairs [0, 22), h [22, 43), w [43, 64)
+          const char *rt = reinterpret_cast<const char *>(p.rope + (size_t)tpos * 128);
+          const char *rh = reinterpret_cast<const char *>(p.rope + (size_t)hpos * 128);
+          const char *rw = reinterpret_cast<const char *>(p.rope + (size_t)wpos * 128);
+          prefetch_l1(rt); prefetch_l1(rt + 128); prefetch_l1(rt + 168);
+          prefetch_l1(rh + 176); prefetch_l1(rh + 296); prefetch_l1(rh + 336);
+          prefetch_l1(rw + 344); prefetch_l1(rw + 464); prefetch_l1(rw + 504);
+        }
+      }
+      if (!mbar_wait(smem_u32(&tfull[buf]), acc_phase, abort_flag, p.watchdog, 0x121)) break;
+      tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         uint32_t r[32];
@@ -379,14 +400,29 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               // [c - 2(c/3), c/3, c/3] pairs, c = head_dim / 2
               const int half = p.head_dim >> 1, c3 = half / 3, pt = half - 2 * c3;
               const int jp0 = (col % p.head_dim) >> 1;
+              // two pairs per load: the entries (pos, jp) and (pos, jp + 1) are
+              // adjacent (16 bytes, jp even); where the two pairs take
+              // different positions (the t/h and h/w borders) they are read
+              // one by one
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int jp = jp0 + e;
-                const int pos = jp < pt ? tpos : (jp < pt + c3 ? hpos : wpos);
-                const float2 cs = *reinterpret_cast<const float2 *>(p.rope + ((size_t)pos * half + jp) * 2);
-                const float x0 = v[2 * e], x1 = v[2 * e + 1];
-                v[2 * e] = x0 * cs.x - x1 * cs.y;
-                v[2 * e + 1] = x0 * cs.y + x1 * cs.x;
+              for (int e2 = 0; e2 < 8; ++e2) {
+                const int jp = jp0 + 2 * e2;
+                const int pa = jp < pt ? tpos : (jp < pt + c3 ? hpos : wpos);
+                const int pb = jp + 1 < pt ? tpos : (jp + 1 < pt + c3 ? hpos : wpos);
+                const float *ra = p.rope + ((size_t)pa * half + jp) * 2;
+                float4 cs;
+                if (pa == pb && p.rope_vec) {
+                  cs = *reinterpret_cast<const float4 *>(ra);
+                } else {
+                  const float2 ca = *reinterpret_cast<const float2 *>(ra);
+                  const float2 cb = *reinterpret_cast<const float2 *>(p.rope + ((size_t)pb * half + jp + 1) * 2);
+                  cs = make_float4(ca.x, ca.y, cb.x, cb.y);
+                }
+                const float x0 = v[4 * e2], x1 = v[4 * e2 + 1], x2 = v[4 * e2 + 2], x3 = v[4 * e2 + 3];
+                v[4 * e2] = x0 * cs.x - x1 * cs.y;
+                v[4 * e2 + 1] = x0 * cs.y + x1 * cs.x;
+                v[4 * e2 + 2] = x2 * cs.z - x3 * cs.w;
+                v[4 * e2 + 3] = x2 * cs.w + x3 * cs.z;
               }
             }
           }
@@ -564,6 +600,7 @@ int gemm_tc(const GemmArgs &g, cudaStream_t s) {
   p.H = g.H > 0 ? g.H : 1; p.W = g.W > 0 ? g.W : 1;
   p.tok0 = g.tok0;
   p.head_dim = g.head_dim > 0 ? g.head_dim : 128;
+  p.rope_vec = aligned16(g.rope) && p.head_dim % 4 == 0;   // 16-byte loads of two table entries
   p.watchdog = watchdog_ptr();
   p.dbg = g.dbg ? g.dbg : dbg_word();
   if (g.ss) p.ss_hi = g.ss + (size_t)g.M * g.ss_stride;
