@@ -39,9 +39,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # same kernel source (sha256 prefix below); reported as null once the source
 # has changed since the capture.
 TRAFFIC = {
-    # profiles/attn_tc_B1_L16384.md: 652.6 MB per launch at B=1, L=16384, scaled by the
+    # profiles/attn_tc_B1_L16384.md: 653.4 MB per launch at B=1, L=16384, scaled by the
     # query/key rows (x4) to the step's launch at B=2, L=32760
-    "attn_self": {"bytes_per_launch": 4 * 652.6e6, "source_sha": "f80a182236bf1ae4"},
+    "attn_self": {"bytes_per_launch": 4 * 653.4e6, "source_sha": "39316987c6657670"},
 }
 
 
