@@ -275,6 +275,16 @@ def test_block_bf16_wide_dims(dim):
     _bf16_block_check(cfg, B=2, ctx_lens=[16, 5])
 
 
+@pytest.mark.parametrize("dim,ffn", [(256, 576), (4096, 4160)])
+def test_block_bf16_ffn_partial_tiles(dim, ffn):
+    """FFN widths that are multiples of 64 but not of 256: the FFN1 GEMM ends in
+    a partial column tile (64 of 256 columns on the narrow tile, K = 256; 64 of
+    512 on the wide tile, K = 4096, whose second column half holds no output at
+    all); the FFN2 GEMM then runs K = 576 / 4160, 9 and 65 K stages of 64."""
+    cfg = BlockConfig(f"bf16-ffn{ffn}", 2, 3, 5, dim, dim // 128, ffn, 16, "bf16")
+    _bf16_block_check(cfg, B=2, ctx_lens=[16, 7])
+
+
 def test_block_1p3b_short():
     _bf16_block_check(configs.get("1.3b-short"))
 
