@@ -294,17 +294,31 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         hpos = (tok / p.W) % p.H;
         wpos = tok % p.W;
       }
-      // the bias, gamma, gate and RoPE-table lines this warp reads go to L1
-      // while the tile's products still run (each would otherwise cost its
-      // chunk an L2 round trip)
+      // Per-column operands, read while the tile's products still run and
+      // spread over the warp: lane l holds columns 8 l .. 8 l + 7 of the warp's
+      // 256 (the bias as 8 bf16; gamma, or the gate row when all 32 rows of
+      // the warp share one, as 8 floats); each chunk takes them by shuffles.
+      const int m0w = mb * 2 * BM + (int)rank * BM + q * 32;       // the warp's first row (warp-uniform)
+      const bool lane_cols = n0 + 8 * lane + 8 <= p.N;
+      uint4 bias8 = make_uint4(0u, 0u, 0u, 0u);
+      float4 col_lo = make_float4(1.f, 1.f, 1.f, 1.f), col_hi = col_lo;
+      if (bias && lane_cols) bias8 = *reinterpret_cast<const uint4 *>(bias + nn0 + 8 * lane);
+      if (EPI == EPI_QKNORM && gam && lane_cols) {
+        col_lo = *reinterpret_cast<const float4 *>(gam + nn0 + 8 * lane);
+        col_hi = *reinterpret_cast<const float4 *>(gam + nn0 + 8 * lane + 4);
+      }
+      bool gate_shared = false;
+      if (EPI == EPI_RESID && p.gate && !p.gate_bias && p.rows_per_gate > 1 && m0w < p.M &&
+          m0w / p.rows_per_gate == min(m0w + 31, p.M - 1) / p.rows_per_gate) {
+        gate_shared = true;
+        if (lane_cols) {
+          const float *gp = p.gate + (size_t)(m0w / p.rows_per_gate) * p.gate_stride + n0 + 8 * lane;
+          col_lo = *reinterpret_cast<const float4 *>(gp);
+          col_hi = *reinterpret_cast<const float4 *>(gp + 4);
+        }
+      }
+      // the RoPE-table lines of this row go to L1 meanwhile
       if (n0 < p.N) {
-        const int last = min(255, p.N - n0 - 1);      // the warp's last column that exists
-        if (bias && lane < 5) prefetch_l1(bias + nn0 + min(lane < 4 ? lane * 64 : 255, last));
-        const float *pf = nullptr;
-        if (EPI == EPI_QKNORM) pf = gam ? gam + nn0 : nullptr;
-        if (EPI == EPI_RESID && p.gate && p.rows_per_gate > 1 && m < p.M)
-          pf = p.gate + (size_t)(m / p.rows_per_gate) * p.gate_stride + n0;
-        if (pf && lane >= 8 && lane < 17) prefetch_l1(pf + min(lane < 16 ? (lane - 8) * 32 : 255, last));
         if (EPI == EPI_QKNORM && do_rope && p.head_dim == 128) {
           // one table row is 64 pairs (512 bytes): t pairs [0, 22), h [22, 43), w [43, 64)
           const char *rt = reinterpret_cast<const char *>(p.rope + (size_t)tpos * 128);
@@ -329,13 +343,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
         const int n = n0 + c * 32;
         // warp-uniform: rows of the warp beyond M are clipped by the tensor map
-        if (mb * 2 * BM + (int)rank * BM + q * 32 >= p.M || n >= p.N) continue;
+        if (m0w >= p.M || n >= p.N) continue;
         float v[32];
-        const uint4 *bp = reinterpret_cast<const uint4 *>(bias + nn0 + c * 32);
+        // column j of the chunk is column 32 c + j of the warp: lane 4 c + j / 8 holds it
 #pragma unroll
         for (int j4 = 0; j4 < 4; ++j4) {
-          const uint4 bb = bias ? bp[j4] : make_uint4(0, 0, 0, 0);
-          const uint32_t w[4] = {bb.x, bb.y, bb.z, bb.w};
+          const uint32_t w[4] = {__shfl_sync(0xffffffffu, bias8.x, 4 * c + j4),
+                                 __shfl_sync(0xffffffffu, bias8.y, 4 * c + j4),
+                                 __shfl_sync(0xffffffffu, bias8.z, 4 * c + j4),
+                                 __shfl_sync(0xffffffffu, bias8.w, 4 * c + j4)};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             if (F8) {
@@ -351,7 +367,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           // x[m, n..n+31] += g * v through a swizzled shared-memory tile and a
           // TMA reduce-add (the read-modify-write of x happens in L2; rows
           // beyond M are clipped by the tensor map)
-          const int m0w = mb * 2 * BM + (int)rank * BM + q * 32;       // warp-uniform
           const float *gr = (p.gate && m < p.M)
                                 ? p.gate + (size_t)(m / p.rows_per_gate) * p.gate_stride + n : nullptr;
           uint8_t *buf = sE + (ew * NSTG + stg_count % NSTG) * STG_BYTES;
@@ -360,7 +375,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
           for (int j16 = 0; j16 < 8; ++j16) {
             float4 gv = make_float4(1.f, 1.f, 1.f, 1.f);
-            if (p.gate) {
+            if (gate_shared) {
+              // columns 4 j16 .. + 3 of the chunk: lane 4 c + j16 / 2, half j16 % 2
+              const int sl = 4 * c + (j16 >> 1);
+              const float4 &src = (j16 & 1) ? col_hi : col_lo;
+              gv = make_float4(__shfl_sync(0xffffffffu, src.x, sl), __shfl_sync(0xffffffffu, src.y, sl),
+                               __shfl_sync(0xffffffffu, src.z, sl), __shfl_sync(0xffffffffu, src.w, sl));
+              if (m >= p.M) gv = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else if (p.gate) {
               gv = gr ? *reinterpret_cast<const float4 *>(gr + 4 * j16) : make_float4(0.f, 0.f, 0.f, 0.f);
               if (p.gate_bias) {
                 const float4 gb = *reinterpret_cast<const float4 *>(p.gate_bias + n + 4 * j16);
@@ -391,8 +413,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             if (gam) {
 #pragma unroll
               for (int j = 0; j < 32; j += 4) {
-                const float4 g4 = *reinterpret_cast<const float4 *>(gam + col + j);
-                v[j] *= g4.x; v[j + 1] *= g4.y; v[j + 2] *= g4.z; v[j + 3] *= g4.w;
+                const int sl = 4 * c + (j >> 3);
+                const float4 &src = (j & 4) ? col_hi : col_lo;
+                v[j] *= __shfl_sync(0xffffffffu, src.x, sl);
+                v[j + 1] *= __shfl_sync(0xffffffffu, src.y, sl);
+                v[j + 2] *= __shfl_sync(0xffffffffu, src.z, sl);
+                v[j + 3] *= __shfl_sync(0xffffffffu, src.w, sl);
               }
             }
             if (do_rope) {
@@ -430,7 +456,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           // 32 x 64 shared-memory tile (128-byte rows, 16-byte chunk k of row r
           // at k ^ (r & 7)) and one TMA store of the tile
           const int sub = c & 1;
-          const int m0w = mb * 2 * BM + (int)rank * BM + q * 32;       // warp-uniform
           uint8_t *sbuf = sE + (ew * NSTG + stg_count % NSTG) * STG_BYTES;
           if (sub == 0) {
             if (lane == 0) bulk_wait_group_read<NSTG - 1>();   // this tile's previous store has read it
